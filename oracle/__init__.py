@@ -1,0 +1,240 @@
+"""CPU oracle for the compression phase of 1-bit Adam (arXiv 2102.02888).
+
+TEST INFRASTRUCTURE ONLY. This package wraps ``onebit_oracle.c``, a plain single-threaded C
+restatement of the method, with ctypes and numpy. Only the test suite, the package's smoke
+check and the benchmark's CPU-baseline leg (and its ``--impl reference`` arm) may import it; the
+product path (the CUDA library and its binding) never does, and the two share no code.
+
+All arrays are numpy, C-contiguous. Grads are float32 ``[W][d]`` or bf16 bit patterns stored as
+uint16 ``[W][d]``. Every function follows the conventions R1-R11 stated at the top of the C
+file; each cites the page and section it restates.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "onebit_oracle.c")
+_LIB = os.path.join(_HERE, "libonebit_oracle.so")
+
+# Flags that keep every fp32 operation a single IEEE operation (R7): no contraction to FMA, no
+# fast-math reassociation; SSE arithmetic on x86-64 has no excess precision.
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+          "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle to ``oracle/libonebit_oracle.so`` (gcc) if missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = _load(build())
+    return _lib
+
+
+def _load(path: str):
+    L = ctypes.CDLL(path)
+    P = ctypes.c_void_p
+    i64, i32, f32, c_int = ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_int
+    L.oracle_pack.argtypes = [P, i64, P]
+    L.oracle_pack.restype = None
+    L.oracle_unpack.argtypes = [P, P, i64, i64, P]
+    L.oracle_unpack.restype = None
+    L.oracle_warmup_step.argtypes = [i64, i32, f32, f32, f32, f32, P, P, P, P, c_int]
+    L.oracle_warmup_step.restype = None
+    L.oracle_worker.argtypes = [i64, i32, i64, f32, P, P, c_int, P, P, P]
+    L.oracle_worker.restype = None
+    L.oracle_server.argtypes = [i64, i32, i64, P, P, P, P, P, P]
+    L.oracle_server.restype = i64
+    L.oracle_apply.argtypes = [i64, i64, f32, f32, P, P, P, P, P]
+    L.oracle_apply.restype = None
+    L.oracle_compressed_step.argtypes = [i64, i32, i64, f32, f32, f32, P, P, P, P, P, P,
+                                         c_int, P, P, P, P, P]
+    L.oracle_compressed_step.restype = i64
+    return L
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _f32(a, shape=None):
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    if shape is not None:
+        assert a.shape == shape, (a.shape, shape)
+    return a
+
+
+def _grads(g: np.ndarray):
+    """Returns (array, gtype): float32 -> 0, uint16 (bf16 bit patterns) -> 1."""
+    if g.dtype == np.float32:
+        return np.ascontiguousarray(g), 0
+    if g.dtype == np.uint16:
+        return np.ascontiguousarray(g), 1
+    raise TypeError("grads must be float32 or uint16 bf16 bit patterns, got %s" % g.dtype)
+
+
+def nchunks(d: int, C: int) -> int:
+    return (d + C - 1) // C
+
+
+def nwords(n: int) -> int:
+    return (n + 31) // 32
+
+
+def pack(x: np.ndarray) -> np.ndarray:
+    """Sign bits of x (bit = x >= 0), LSB-first into uint32 words; padding bits are 0 (R3, R4)."""
+    x = _f32(x).ravel()
+    words = np.zeros(nwords(x.size), dtype=np.uint32)
+    lib().oracle_pack(_p(x), x.size, _p(words))
+    return words
+
+
+def unpack(words: np.ndarray, scales: np.ndarray, n: int, C: int) -> np.ndarray:
+    """Decompression: +-scales[i // C] by the sign bit of element i."""
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    scales = _f32(scales)
+    assert words.size >= nwords(n) and scales.size >= nchunks(n, C)
+    out = np.empty(n, dtype=np.float32)
+    lib().oracle_unpack(_p(words), _p(scales), n, C, _p(out))
+    return out
+
+
+def warmup_step(x, m, v, g, beta1, beta2, eps, lr):
+    """Full-precision Adam warm-up step, in place on x, m, v (no bias correction, R6)."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    for a in (x, m, v):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    lib().oracle_warmup_step(d, W, beta1, beta2, eps, lr, _p(x), _p(m), _p(v), _p(g), gt)
+
+
+def worker(m, g, e_w, C, beta1):
+    """Worker compression for all W workers; e_w ([W][d], explicit) is updated in place.
+
+    Returns (s [W][nch] float32, bits_w [W][ceil(d/32)] uint32)."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    assert e_w.dtype == np.float32 and e_w.shape == (W, d) and e_w.flags["C_CONTIGUOUS"]
+    m = _f32(m, (d,))
+    s = np.zeros((W, nchunks(d, C)), dtype=np.float32)
+    bits = np.zeros((W, nwords(d)), dtype=np.uint32)
+    lib().oracle_worker(d, W, C, beta1, _p(m), _p(g), gt, _p(e_w), _p(s), _p(bits))
+    return s, bits
+
+
+def server(s, bits_w, e_s, C):
+    """Server stage of the compressed allreduce; e_s ([d], explicit) is updated in place.
+
+    Returns (S [nch] float32, bits_s [ceil(d/32)] uint32, z [d] float32, inexact_chunks)."""
+    s = _f32(s)
+    W, nch = s.shape
+    d = e_s.size
+    assert e_s.dtype == np.float32 and e_s.flags["C_CONTIGUOUS"]
+    bits_w = np.ascontiguousarray(bits_w, dtype=np.uint32)
+    assert bits_w.shape == (W, nwords(d)) and nch == nchunks(d, C)
+    S = np.zeros(nch, dtype=np.float32)
+    bits_s = np.zeros(nwords(d), dtype=np.uint32)
+    z = np.zeros(d, dtype=np.float32)
+    inexact = lib().oracle_server(d, W, C, _p(s), _p(bits_w), _p(e_s), _p(z), _p(S), _p(bits_s))
+    return S, bits_s, z, int(inexact)
+
+
+def apply(bits_s, S, v, m, x, C, eps, lr):
+    """m = +-S by the server bits; x -= lr * (m / (sqrt(v) + eps)); in place on m and x."""
+    d = x.size
+    bits_s = np.ascontiguousarray(bits_s, dtype=np.uint32)
+    S = _f32(S)
+    v = _f32(v, (d,))
+    for a in (m, x):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    lib().oracle_apply(d, C, eps, lr, _p(bits_s), _p(S), _p(v), _p(m), _p(x))
+
+
+def compressed_step(x, m, v, e_w, e_s, g, C, beta1, eps, lr):
+    """One whole compressed step, in place on x, m, e_w, e_s (v is read only).
+
+    Returns a dict with the step's messages: s, S, bits_w, bits_s, inexact."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    for a in (x, m, e_s):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    assert e_w.dtype == np.float32 and e_w.shape == (W, d) and e_w.flags["C_CONTIGUOUS"]
+    v = _f32(v, (d,))
+    nch = nchunks(d, C)
+    s = np.zeros((W, nch), dtype=np.float32)
+    S = np.zeros(nch, dtype=np.float32)
+    bits_w = np.zeros((W, nwords(d)), dtype=np.uint32)
+    bits_s = np.zeros(nwords(d), dtype=np.uint32)
+    z = np.zeros(d, dtype=np.float32)
+    inexact = lib().oracle_compressed_step(d, W, C, beta1, eps, lr, _p(x), _p(m), _p(v), _p(e_w),
+                                           _p(e_s), _p(g), gt, _p(s), _p(S), _p(bits_w),
+                                           _p(bits_s), _p(z))
+    return {"s": s, "S": S, "bits_w": bits_w, "bits_s": bits_s, "inexact": int(inexact)}
+
+
+class OracleState:
+    """The optimizer state of the method, held on the host: x, m, v and, after the freeze, the
+    explicit worker and server residuals. Mirrors the phases of the method: warm-up steps, the
+    variance freeze, compressed steps."""
+
+    def __init__(self, x, W, C, beta1=0.9, beta2=0.999, eps=1e-8):
+        self.x = _f32(x).copy()
+        d = self.x.size
+        self.d, self.W, self.C = d, W, C
+        self.beta1, self.beta2, self.eps = beta1, beta2, eps
+        self.m = np.zeros(d, dtype=np.float32)
+        self.v = np.zeros(d, dtype=np.float32)
+        self.e_w = None
+        self.e_s = None
+        self.frozen = False
+
+    def warmup_step(self, g, lr):
+        assert not self.frozen
+        warmup_step(self.x, self.m, self.v, g, self.beta1, self.beta2, self.eps, lr)
+
+    def freeze(self):
+        """Freeze v as the preconditioner; residuals start at zero (R11)."""
+        self.frozen = True
+        self.e_w = np.zeros((self.W, self.d), dtype=np.float32)
+        self.e_s = np.zeros(self.d, dtype=np.float32)
+
+    def compressed_step(self, g, lr):
+        assert self.frozen
+        return compressed_step(self.x, self.m, self.v, self.e_w, self.e_s, g, self.C,
+                               self.beta1, self.eps, lr)
+
+
+class use_library:
+    """Context manager that routes every oracle call through another build of the C file (the
+    test suite uses it to plant mistakes in a copy of the oracle and check its pins catch them)."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
