@@ -1,0 +1,385 @@
+"""Benchmark of the compressed step of 1-bit Adam on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One STEP is one whole compressed step (worker compression of all W workers, the compressed
+allreduce's server stage, the frozen-variance apply) over the workload's parameter bucket, with
+its inputs resident in HBM. The default workload is the BERT-Large-shaped bucket (333,563,904
+fp32 parameters, W = 16 simulated workers, C = d/W, bf16 gradients). The metric is
+params x workers / s of the compressed step, with achieved HBM GB/s against the measured copy
+bandwidth. With N > 1 (torchrun, one process per GPU) every rank runs its own replica of the
+whole workload (the method's W workers are simulated inside each GPU; there is no data-path
+collective) and the value is the sum over ranks, timed as the max over ranks.
+
+``--impl reference`` times the CPU oracle (plain single-threaded C) on a bounded sample of the
+same workload; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "worker_kernel_bert_large_bucket.md")
+KERNEL_SRC = os.path.join(ROOT, "communication_compressed_optimizer_momentum_b200", "csrc",
+                          "kernels.cuh")
+FALLBACK_HBM_GBS = 6650.0
+METRIC = "compressed-step params×workers/sec and achieved HBM GB/s (% of B200 peak)"
+UNIT = "params*workers/s"
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="bert_large_bucket")
+    p.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="CPU time budget of the oracle baseline sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--scale-d", type=int, default=0,
+                   help="run the workload's distributions on a smaller vector (profiling)")
+    return p.parse_args()
+
+
+def get_workload(name, scale_d=0):
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+    if name in wls.WORKLOADS:
+        wl = wls.WORKLOADS[name]
+        return wls.scaled(wl, scale_d) if scale_d else wl
+    if name.startswith("sweep_W"):
+        # sweep_W<w>_C<c>, c = 0 for d/W
+        w, c = name[len("sweep_W"):].split("_C")
+        return wls.sweep_workload(int(w), int(c) or None)
+    raise SystemExit("unknown workload %s" % name)
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha():
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def ncu_traffic(workload):
+    """DRAM bytes per worker-kernel launch from the committed ncu summary, if it was taken on
+    the current kernel source for this workload; otherwise None."""
+    try:
+        with open(PROFILE_SUMMARY) as f:
+            text = f.read()
+    except OSError:
+        return None
+    fields = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_sha():
+        return None
+    if fields.get("workload") != workload:
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch_full"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms in a background process."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append((t, float(parts[2]), float(parts[3]), parts[5:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.2 <= r[0] <= self.t1 + 0.2]
+        use = inside or rows
+        sm = sorted(r[1] for r in use)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in use:
+            for nm, flag in zip(names, r[3][1:5]):
+                if flag.strip().lower() in ("active", "1"):
+                    reasons.add(nm)
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(reasons), "samples": len(use),
+                "in_timed_region": bool(inside)}
+
+
+def _to_np(t):
+    import numpy as np
+    import torch
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16).copy()
+    return t.numpy().copy()
+
+
+def oracle_sample_rate(wl, state, g, seconds):
+    """Time oracle compressed steps on one chunk-sized problem until `seconds` have passed
+    (at least one step). Returns (params*workers/s, steps, elements per step)."""
+    import oracle
+    x, m, v, e_w, e_s = (state[k].copy() for k in ("x", "m", "v", "e_w", "e_s"))
+    n = x.size
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle.compressed_step(x, m, v, e_w, e_s, g, min(wl.C, n), wl.beta1, wl.eps, wl.lr)
+        steps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return steps * n * wl.W / el, steps, n
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import communication_compressed_optimizer_momentum_b200 as ob
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = get_workload(args.workload, args.scale_d)
+    dt = wls.torch_dtype(wl)
+
+    x = wls.torch_params(wl, dev)
+    g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
+    opt = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt, device=dev)
+    for t in range(wl.warmup_steps):             # full-precision Adam warm-up (setup)
+        wls.torch_fill_grads(wl, g, 0, t)
+        opt.warmup_step(x, g, wl.lr)
+    opt.freeze()
+    wls.torch_fill_grads(wl, g, 1, 1)            # resident inputs for the timed steps
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 0)):
+        opt.step(x, g, wl.lr)
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.5)
+    opt.timing(args.steps)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("t0")
+    t_start.record(stream)
+    for _ in range(args.steps):
+        opt.step(x, g, wl.lr)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    kernel_ms, nrec = opt.timing_read()
+    opt.timing(0)
+    time.sleep(0.3)
+    clocks = sampler.stop()
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    status = opt.status()
+
+    units = wl.d * wl.W * args.steps * world
+    value = units / (ms_max / 1e3)
+    step_bytes = wl.algorithmic_bytes_per_param() * wl.d
+    achieved_step_gbs = step_bytes * args.steps / (ms_max / 1e3) / 1e9
+    peak, peak_src = measured_hbm_peak()
+    kb = wl.kernel_bytes_per_param()
+    worker_bytes = kb["worker"] * wl.d
+    worker_ms = kernel_ms["worker"] / max(nrec, 1)
+    worker_gbs = worker_bytes / (worker_ms / 1e3) / 1e9 if worker_ms > 0 else None
+
+    # end to end through the host-buffer entry point: H2D grads, the step, D2H x
+    e2e = None
+    if not args.no_e2e and args.e2e_steps > 0:
+        g_host = torch.empty((wl.W, wl.d), dtype=dt, pin_memory=True)
+        g_host.copy_(g)
+        x_host = torch.empty(wl.d, dtype=torch.float32, pin_memory=True)
+        opt.step_host(x, g, g_host, x_host, wl.lr)      # untimed first call
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            opt.step_host(x, g, g_host, x_host, wl.lr)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e2e = {"value": wl.d * wl.W * args.e2e_steps * world / (float(e_ms.item()) / 1e3),
+               "unit": UNIT, "steps": args.e2e_steps,
+               "h2d_bytes_per_step": wl.W * wl.d * wl.grad_bytes,
+               "d2h_bytes_per_step": wl.d * 4}
+        del g_host, x_host
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        k = 0
+        lo, hi = 0, min(wl.d, wl.C)
+        st = {"x": _to_np(x[lo:hi]), "m": _to_np(opt.get_chunk_state("m", k)),
+              "v": _to_np(opt.get_chunk_state("v", k)),
+              "e_w": _to_np(opt.get_chunk_state("e_w", k)),
+              "e_s": _to_np(opt.get_chunk_state("e_s", k))}
+        gk = _to_np(g[:, lo:hi])
+        rate, n_steps, n = oracle_sample_rate(wl, st, gk, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": "chunk 0 of the workload (%d params x %d workers), %d oracle "
+                         "compressed step(s), single-threaded C" % (n, wl.W, n_steps)}
+
+    if rank == 0:
+        from communication_compressed_optimizer_momentum_b200 import workloads as _w
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": dict(_w.describe(wl), parallelism="replicas" if world > 1 else "single",
+                           l2="inputs larger than L2 (%.1f GB resident); no flush" % (
+                               (opt.workspace_bytes + wl.W * wl.d * wl.grad_bytes
+                                + wl.d * 4) / 1e9),
+                           grads_resident="one seeded draw reused by every timed step"),
+            "achieved_hbm_gbs": achieved_step_gbs,
+            "pct_of_hbm_peak": 100.0 * achieved_step_gbs / peak,
+            "algorithmic_bytes_per_step": step_bytes,
+            "kernel_ms_per_step": {k2: v2 / max(nrec, 1) for k2, v2 in kernel_ms.items()},
+            "roofline": {"bound": "hbm", "kernel": "worker", "achieved": worker_gbs,
+                         "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                         "frac": (worker_gbs / peak) if worker_gbs else None,
+                         "traffic": ncu_traffic(wl.name),
+                         "algorithmic_bytes_per_launch": worker_bytes},
+            "gpu_launches": opt.info()["launches_per_step"] * args.steps,
+            "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "status_flags": status,
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands on the host cores, on a bounded sample of the same workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+    wl = get_workload(args.workload)
+    n = min(wl.d, 1 << 20)
+    sw = wls.scaled(wl, n, C=min(wl.C, n))
+    x = wls.np_params(sw)
+    st = oracle.OracleState(x, sw.W, sw.C, sw.beta1, sw.beta2, sw.eps)
+    st.warmup_step(wls.np_grads(sw, 0, 0), sw.lr)
+    st.freeze()
+    g = wls.np_grads(sw, 1, 1)
+    for _ in range(max(args.warmup, 0)):
+        st.compressed_step(g, sw.lr)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        st.compressed_step(g, sw.lr)
+    el = time.perf_counter() - t0
+    value = n * sw.W * args.steps / el
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "impl": "reference",
+        "config": dict(wls.describe(wl), sample_d=n, sample_C=sw.C),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "%d params x %d workers (one chunk) of %s per step, "
+                                   "single-threaded C oracle" % (n, sw.W, wl.name)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,283 @@
+"""1-bit Adam compression phase on B200: Python binding of the C ABI (``include/onebit_adam.h``).
+
+Every function below has the name of the C entry point it wraps and does argument marshalling
+only (tensor -> device pointer, stream -> cudaStream_t, status code -> exception). All the
+arithmetic of the method runs in the library's CUDA kernels; torch provides device memory and
+streams. There is no CPU fallback: if the library is missing or the call fails, an exception is
+raised.
+
+``OneBitAdam`` is a small convenience owner of one handle and its torch-allocated workspace.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+from . import _abi
+
+ONEBIT_F32, ONEBIT_BF16 = 0, 1
+STATE = {"m": 0, "v": 1, "e_w": 2, "e_s": 3, "s": 4, "S": 5, "bits_w": 6, "bits_s": 7}
+FLAG_NAN_WORKER, FLAG_NAN_SERVER = 1, 2
+KERNELS = ("worker", "worker_scales", "server", "server_scales", "apply")
+
+
+class OneBitError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        L = _abi.lib()
+        msg = L.onebit_strerror(code).decode()
+        extra = L.onebit_last_error().decode() if code == -4 else ""
+        super().__init__("%s failed: %s (%d)%s" % (where, msg, code, (": " + extra) if extra else ""))
+        self.code = code
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise OneBitError(rc, where)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(None)
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(dtype) -> int:
+    import torch
+    if dtype == torch.float32:
+        return ONEBIT_F32
+    if dtype == torch.bfloat16:
+        return ONEBIT_BF16
+    raise TypeError("gradients must be float32 or bfloat16, got %s" % dtype)
+
+
+def _handle(h) -> ctypes.c_void_p:
+    return h if isinstance(h, ctypes.c_void_p) else ctypes.c_void_p(h)
+
+
+# ----------------------------------------------------------------------------------------------
+# the C entry points
+
+def onebit_adam_init(d: int, W: int, C: int, beta1: float = 0.9, beta2: float = 0.999,
+                     eps: float = 1e-8) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_abi.lib().onebit_adam_init(ctypes.byref(h), d, W, C, beta1, beta2, eps),
+           "onebit_adam_init")
+    return h
+
+
+def onebit_adam_workspace_bytes(h, grad_dtype: int) -> int:
+    n = ctypes.c_uint64()
+    _check(_abi.lib().onebit_adam_workspace_bytes(_handle(h), grad_dtype, ctypes.byref(n)),
+           "onebit_adam_workspace_bytes")
+    return n.value
+
+
+def onebit_adam_bind(h, workspace, nbytes: int, grad_dtype: int, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_bind(_handle(h), _ptr(workspace), nbytes, grad_dtype,
+                                       _stream(stream)), "onebit_adam_bind")
+
+
+def onebit_adam_warmup_step(h, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_warmup_step(_handle(h), _ptr(x), _ptr(grads), lr,
+                                              _stream(stream)), "onebit_adam_warmup_step")
+
+
+def onebit_adam_freeze_variance(h, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_freeze_variance(_handle(h), _stream(stream)),
+           "onebit_adam_freeze_variance")
+
+
+def onebit_adam_compressed_step(h, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_compressed_step(_handle(h), _ptr(x), _ptr(grads), lr,
+                                                  _stream(stream)),
+           "onebit_adam_compressed_step")
+
+
+def onebit_adam_compressed_step_host(h, x_dev, grads_dev, grads_host, x_host, lr: float,
+                                     stream=None) -> None:
+    _check(_abi.lib().onebit_adam_compressed_step_host(
+        _handle(h), _ptr(x_dev), _ptr(grads_dev), _ptr(grads_host), _ptr(x_host), lr,
+        _stream(stream)), "onebit_adam_compressed_step_host")
+
+
+def onebit_adam_state_bytes(h, which: int) -> int:
+    n = ctypes.c_uint64()
+    _check(_abi.lib().onebit_adam_state_bytes(_handle(h), which, ctypes.byref(n)),
+           "onebit_adam_state_bytes")
+    return n.value
+
+
+def onebit_adam_get_state(h, which: int, dst, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_get_state(_handle(h), which, _ptr(dst), _stream(stream)),
+           "onebit_adam_get_state")
+
+
+def onebit_adam_get_chunk_state(h, which: int, k: int, dst, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_get_chunk_state(_handle(h), which, k, _ptr(dst),
+                                                  _stream(stream)),
+           "onebit_adam_get_chunk_state")
+
+
+def onebit_adam_set_state(h, which: int, src, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_set_state(_handle(h), which, _ptr(src), _stream(stream)),
+           "onebit_adam_set_state")
+
+
+def onebit_adam_status(h, stream=None) -> int:
+    f = ctypes.c_uint32()
+    _check(_abi.lib().onebit_adam_status(_handle(h), _stream(stream), ctypes.byref(f)),
+           "onebit_adam_status")
+    return f.value
+
+
+def onebit_adam_info(h) -> dict:
+    out = (ctypes.c_int64 * 8)()
+    _check(_abi.lib().onebit_adam_info(_handle(h), out), "onebit_adam_info")
+    keys = ("d", "W", "C", "nch", "phase", "steps", "grad_dtype", "launches_per_step")
+    return dict(zip(keys, list(out)))
+
+
+def onebit_adam_timing(h, max_steps: int) -> None:
+    _check(_abi.lib().onebit_adam_timing(_handle(h), max_steps), "onebit_adam_timing")
+
+
+def onebit_adam_timing_read(h) -> Tuple[dict, int]:
+    ms = (ctypes.c_double * 5)()
+    n = ctypes.c_int32()
+    _check(_abi.lib().onebit_adam_timing_read(_handle(h), ms, ctypes.byref(n)),
+           "onebit_adam_timing_read")
+    return dict(zip(KERNELS, list(ms))), n.value
+
+
+def onebit_adam_destroy(h) -> None:
+    _abi.lib().onebit_adam_destroy(_handle(h))
+
+
+def onebit_strerror(code: int) -> str:
+    return _abi.lib().onebit_strerror(code).decode()
+
+
+def onebit_last_error() -> str:
+    return _abi.lib().onebit_last_error().decode()
+
+
+def onebit_pack(x, words=None, stream=None):
+    """Sign-pack a contiguous float32 CUDA tensor into int32 words (LSB-first)."""
+    import torch
+    n = x.numel()
+    if words is None:
+        words = torch.empty((n + 31) // 32, dtype=torch.int32, device=x.device)
+    _check(_abi.lib().onebit_pack(_ptr(x), n, _ptr(words), _stream(stream)), "onebit_pack")
+    return words
+
+
+def onebit_unpack(words, scales, n: int, C: int, out=None, stream=None):
+    """Decompress packed words with per-chunk scales into a float32 CUDA tensor."""
+    import torch
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=words.device)
+    _check(_abi.lib().onebit_unpack(_ptr(words), _ptr(scales), n, C, _ptr(out), _stream(stream)),
+           "onebit_unpack")
+    return out
+
+
+# ----------------------------------------------------------------------------------------------
+# convenience owner of one handle + workspace
+
+class OneBitAdam:
+    """One optimizer instance: the handle plus its device workspace (allocated with torch).
+
+    Phases follow the method: ``warmup_step`` (full-precision Adam) any number of times, then
+    ``freeze()`` (the variance becomes the fixed preconditioner), then ``step`` (compressed)."""
+
+    def __init__(self, d: int, W: int, C: int, beta1: float = 0.9, beta2: float = 0.999,
+                 eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None):
+        import torch
+        grad_dtype = torch.float32 if grad_dtype is None else grad_dtype
+        self.d, self.W, self.C = d, W, C
+        self.grad_dtype = grad_dtype
+        self.h = onebit_adam_init(d, W, C, beta1, beta2, eps)
+        code = dtype_code(grad_dtype)
+        nbytes = onebit_adam_workspace_bytes(self.h, code)
+        raw = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)
+        shift = (-raw.data_ptr()) % 256
+        self._raw = raw
+        self.workspace = raw[shift:shift + nbytes]
+        self.workspace_bytes = nbytes
+        onebit_adam_bind(self.h, self.workspace, nbytes, code, stream)
+        self.nch = (d + C - 1) // C
+
+    def warmup_step(self, x, grads, lr: float, stream=None) -> None:
+        onebit_adam_warmup_step(self.h, x, grads, lr, stream)
+
+    def freeze(self, stream=None) -> None:
+        onebit_adam_freeze_variance(self.h, stream)
+
+    def step(self, x, grads, lr: float, stream=None) -> None:
+        onebit_adam_compressed_step(self.h, x, grads, lr, stream)
+
+    def step_host(self, x_dev, grads_dev, grads_host, x_host, lr: float, stream=None) -> None:
+        onebit_adam_compressed_step_host(self.h, x_dev, grads_dev, grads_host, x_host, lr, stream)
+
+    def state_shape(self, which: str):
+        d, W, nch, nw = self.d, self.W, self.nch, (self.d + 31) // 32
+        return {"m": (d,), "v": (d,), "e_w": (W, d), "e_s": (d,), "s": (W, nch), "S": (nch,),
+                "bits_w": (W, nw), "bits_s": (nw,)}[which]
+
+    def get_state(self, which: str, stream=None):
+        import torch
+        dt = torch.int32 if which.startswith("bits") else torch.float32
+        out = torch.empty(self.state_shape(which), dtype=dt, device=self.workspace.device)
+        onebit_adam_get_state(self.h, STATE[which], out, stream)
+        return out
+
+    def chunk_shape(self, which: str, k: int):
+        n = min(self.C, self.d - k * self.C)
+        nwk = (n + 31) // 32
+        return {"m": (n,), "v": (n,), "e_w": (self.W, n), "e_s": (n,), "s": (self.W,),
+                "S": (1,), "bits_w": (self.W, nwk), "bits_s": (nwk,)}[which]
+
+    def get_chunk_state(self, which: str, k: int, stream=None):
+        import torch
+        dt = torch.int32 if which.startswith("bits") else torch.float32
+        out = torch.empty(self.chunk_shape(which, k), dtype=dt, device=self.workspace.device)
+        onebit_adam_get_chunk_state(self.h, STATE[which], k, out, stream)
+        return out
+
+    def set_state(self, which: str, src, stream=None) -> None:
+        assert tuple(src.shape) == self.state_shape(which) and src.is_contiguous()
+        onebit_adam_set_state(self.h, STATE[which], src, stream)
+
+    def status(self, stream=None) -> int:
+        return onebit_adam_status(self.h, stream)
+
+    def info(self) -> dict:
+        return onebit_adam_info(self.h)
+
+    def timing(self, max_steps: int) -> None:
+        onebit_adam_timing(self.h, max_steps)
+
+    def timing_read(self):
+        return onebit_adam_timing_read(self.h)
+
+    def close(self) -> None:
+        if getattr(self, "h", None) is not None:
+            onebit_adam_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

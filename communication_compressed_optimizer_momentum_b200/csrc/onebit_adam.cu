@@ -1,0 +1,571 @@
+// onebit_adam.cu -- host side of the C ABI declared in include/onebit_adam.h: argument checks,
+// the workspace layout, the launch sequence of one step and the state/timing helpers.
+//
+// One compressed step is five launches on the caller's stream, ordered by the stream alone
+// (no kernel waits on another, so nothing can spin or hang):
+//   k_worker  -> k_scales (worker)  -> k_server -> k_scales (server) -> k_apply
+// The boundary between k_worker/k_scales and k_server is where the compressed allreduce of the
+// method crosses the network ("1-bit Adam" index page, Abstract: communication is the
+// bottleneck; LIT-278 note: the compressed allreduce is a custom collective); here the W
+// workers live in one GPU's memory, so the "network" is the packed planes in HBM.
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "onebit_adam.h"
+#include "kernels.cuh"
+
+using namespace onebit;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+constexpr int32_t kMaxWorkers = 256;
+constexpr int kLaunchesPerStep = 5;
+constexpr int kEventsPerStep = kLaunchesPerStep + 1;
+
+enum Phase { kUnbound = 0, kWarmup = 1, kCompressed = 2 };
+
+int cuda_fail(cudaError_t e) {
+    g_last_error = cudaGetErrorString(e);
+    return ONEBIT_ERR_CUDA;
+}
+
+#define ONEBIT_CUDA(call)                                 \
+    do {                                                  \
+        cudaError_t e_ = (call);                          \
+        if (e_ != cudaSuccess) return cuda_fail(e_);      \
+    } while (0)
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Workspace regions, each 256-byte aligned.
+struct Layout {
+    uint64_t m, v, es, ew, bits_w, bits_s, s_out, s_lazy, S_out, S_lazy, part_w, part_s, status;
+    uint64_t total;
+};
+
+}  // namespace
+
+struct onebit_adam_s {
+    Geometry geo;
+    int64_t nw;  // words per plane, ceil(d / 32)
+    float beta1, beta2, eps;
+    int phase = kUnbound;
+    int64_t steps = 0;
+    int32_t gtype = -1;
+    char* ws = nullptr;
+    Layout lay{};
+    // region pointers (valid once bound)
+    float *m = nullptr, *v = nullptr, *es = nullptr, *ew = nullptr;
+    float *s_out = nullptr, *s_lazy = nullptr, *S_out = nullptr, *S_lazy = nullptr;
+    uint32_t *bits_w = nullptr, *bits_s = nullptr, *status = nullptr;
+    double *part_w = nullptr, *part_s = nullptr;
+    // per-kernel timing
+    std::vector<cudaEvent_t> ev;
+    int32_t tmax = 0, tcount = 0;
+};
+
+namespace {
+
+Layout make_layout(const onebit_adam_s& h) {
+    const Geometry& g = h.geo;
+    Layout L{};
+    uint64_t off = 0;
+    auto take = [&](uint64_t bytes) {
+        const uint64_t at = off;
+        off = (uint64_t)round_up((int64_t)(off + bytes), 256);
+        return at;
+    };
+    const uint64_t f = sizeof(float);
+    L.m = take(g.ld * f);
+    L.v = take(g.ld * f);
+    L.es = take(g.ld * f);
+    L.ew = take((uint64_t)g.W * g.ld * f);
+    L.bits_w = take((uint64_t)g.W * g.ldw * sizeof(uint32_t));
+    L.bits_s = take(g.ldw * sizeof(uint32_t));
+    L.s_out = take((uint64_t)g.W * g.nch * f);
+    L.s_lazy = take((uint64_t)g.W * g.nch * f);
+    L.S_out = take(g.nch * f);
+    L.S_lazy = take(g.nch * f);
+    L.part_w = take((uint64_t)g.W * g.nch * g.nseg * sizeof(double));
+    L.part_s = take((uint64_t)g.nch * g.nseg * sizeof(double));
+    L.status = take(4 * sizeof(uint32_t));
+    L.total = off;
+    return L;
+}
+
+bool valid_handle(onebit_adam_t h) { return h != nullptr; }
+
+int64_t step_blocks(const Geometry& g) { return g.nch * g.nseg; }
+
+// Launch the chunk-scale reduction with the thread count that fits the partial count.
+int launch_scales(const Geometry& g, const double* part, int64_t rows, float* out, float* lazy,
+                  cudaStream_t st) {
+    if (rows == 0) return ONEBIT_OK;
+    if (g.nseg <= 8) {
+        k_scales<1><<<(unsigned)ceil_div(rows, kThreads), kThreads, 0, st>>>(
+            part, rows, g.nch, g.nseg, g.C, g.d, out, lazy);
+    } else if (g.nseg <= 1024) {
+        k_scales<32><<<(unsigned)ceil_div(rows, kWarps), kThreads, 0, st>>>(
+            part, rows, g.nch, g.nseg, g.C, g.d, out, lazy);
+    } else {
+        k_scales<kThreads><<<(unsigned)rows, kThreads, 0, st>>>(part, rows, g.nch, g.nseg, g.C,
+                                                                g.d, out, lazy);
+    }
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+template <typename GT>
+int launch_worker(onebit_adam_s* h, const void* grads, cudaStream_t st) {
+    WorkerArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->m, grads, h->ew, h->s_lazy, h->bits_w,
+                 h->part_w, h->status};
+    const size_t smem = (size_t)h->geo.W * kWarps * sizeof(double);
+    const unsigned blocks = (unsigned)step_blocks(h->geo);
+    if (h->geo.d % kVec == 0)
+        k_worker<GT, true><<<blocks, kThreads, smem, st>>>(a);
+    else
+        k_worker<GT, false><<<blocks, kThreads, smem, st>>>(a);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+template <typename GT>
+int launch_warmup(onebit_adam_s* h, float* x, const void* grads, float lr, cudaStream_t st) {
+    WarmupArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->beta2, 1.0f - h->beta2, h->eps, lr,
+                 grads, h->m, h->v, x};
+    const unsigned blocks = (unsigned)step_blocks(h->geo);
+    if (h->geo.d % kVec == 0)
+        k_warmup<GT, true><<<blocks, kThreads, 0, st>>>(a);
+    else
+        k_warmup<GT, false><<<blocks, kThreads, 0, st>>>(a);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+void record(onebit_adam_s* h, int slot, cudaStream_t st) {
+    if (h->tcount < h->tmax) cudaEventRecord(h->ev[(size_t)h->tcount * kEventsPerStep + slot], st);
+}
+
+void free_events(onebit_adam_s* h) {
+    for (cudaEvent_t e : h->ev) cudaEventDestroy(e);
+    h->ev.clear();
+    h->tmax = h->tcount = 0;
+}
+
+uint64_t grad_elem_bytes(int32_t gtype) { return gtype == ONEBIT_BF16 ? 2 : 4; }
+
+// Explicit residuals of elements [i0, i0 + n) of every row (W rows for the workers, 1 for the
+// server) into dst[rows][n].
+int launch_materialize(onebit_adam_s* h, bool workers, int64_t i0, int64_t n, float* dst,
+                       cudaStream_t st) {
+    const Geometry& g = h->geo;
+    const int64_t rows = workers ? g.W : 1;
+    const int64_t total = rows * n;
+    if (total == 0) return ONEBIT_OK;
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(total, kThreads), 148 * 32);
+    k_materialize<<<blocks, kThreads, 0, st>>>(workers ? h->ew : h->es, g.ld,
+                                               workers ? h->s_lazy : h->S_lazy, g.nch, g.C, i0,
+                                               n, rows, dst);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* onebit_strerror(int32_t code) {
+    switch (code) {
+        case ONEBIT_OK: return "ok";
+        case ONEBIT_ERR_ARG: return "invalid argument";
+        case ONEBIT_ERR_ALIGN: return "misaligned pointer or chunk length not a multiple of 32";
+        case ONEBIT_ERR_PHASE: return "call not allowed in the handle's current phase";
+        case ONEBIT_ERR_CUDA: return "CUDA error";
+        case ONEBIT_ERR_SPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+const char* onebit_last_error(void) { return g_last_error.c_str(); }
+
+int onebit_adam_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                     float beta2, float eps) {
+    if (out == nullptr) return ONEBIT_ERR_ARG;
+    *out = nullptr;
+    if (d < 0 || W < 1 || W > kMaxWorkers || C <= 0) return ONEBIT_ERR_ARG;
+    if (C % 32 != 0) return ONEBIT_ERR_ALIGN;
+    if (!std::isfinite(beta1) || !std::isfinite(beta2) || !std::isfinite(eps)) return ONEBIT_ERR_ARG;
+    if (beta1 < 0.0f || beta1 >= 1.0f || beta2 < 0.0f || beta2 >= 1.0f || eps < 0.0f)
+        return ONEBIT_ERR_ARG;
+    // sizes must stay far from int64 overflow: W * ld * 8 bytes < 2^62
+    if (d > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
+    onebit_adam_s* h = new (std::nothrow) onebit_adam_s();
+    if (h == nullptr) return ONEBIT_ERR_ARG;
+    Geometry& g = h->geo;
+    g.d = d;
+    g.W = W;
+    g.C = C;
+    g.nch = ceil_div(d, C);
+    g.nseg = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSeg);
+    g.ld = round_up(d > 0 ? d : 1, 64);
+    h->nw = ceil_div(d, 32);
+    g.ldw = round_up(h->nw > 0 ? h->nw : 1, 4);
+    h->beta1 = beta1;
+    h->beta2 = beta2;
+    h->eps = eps;
+    if (g.nch * g.nseg > (int64_t)INT32_MAX) {  // one block per segment must fit the grid
+        delete h;
+        return ONEBIT_ERR_ARG;
+    }
+    *out = h;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_workspace_bytes(onebit_adam_t h, int32_t grad_dtype, uint64_t* bytes) {
+    if (!valid_handle(h) || bytes == nullptr) return ONEBIT_ERR_ARG;
+    if (grad_dtype != ONEBIT_F32 && grad_dtype != ONEBIT_BF16) return ONEBIT_ERR_ARG;
+    *bytes = make_layout(*h).total;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t grad_dtype,
+                     void* stream) {
+    if (!valid_handle(h) || workspace == nullptr) return ONEBIT_ERR_ARG;
+    if (grad_dtype != ONEBIT_F32 && grad_dtype != ONEBIT_BF16) return ONEBIT_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ONEBIT_ERR_ALIGN;
+    const Layout L = make_layout(*h);
+    if (bytes < L.total) return ONEBIT_ERR_SPACE;
+    char* b = static_cast<char*>(workspace);
+    h->ws = b;
+    h->lay = L;
+    h->m = reinterpret_cast<float*>(b + L.m);
+    h->v = reinterpret_cast<float*>(b + L.v);
+    h->es = reinterpret_cast<float*>(b + L.es);
+    h->ew = reinterpret_cast<float*>(b + L.ew);
+    h->bits_w = reinterpret_cast<uint32_t*>(b + L.bits_w);
+    h->bits_s = reinterpret_cast<uint32_t*>(b + L.bits_s);
+    h->s_out = reinterpret_cast<float*>(b + L.s_out);
+    h->s_lazy = reinterpret_cast<float*>(b + L.s_lazy);
+    h->S_out = reinterpret_cast<float*>(b + L.S_out);
+    h->S_lazy = reinterpret_cast<float*>(b + L.S_lazy);
+    h->part_w = reinterpret_cast<double*>(b + L.part_w);
+    h->part_s = reinterpret_cast<double*>(b + L.part_s);
+    h->status = reinterpret_cast<uint32_t*>(b + L.status);
+    h->gtype = grad_dtype;
+    cudaStream_t st = as_stream(stream);
+    // m and v start at zero (Adam); the rest is cleared too so padding is deterministic.
+    ONEBIT_CUDA(cudaMemsetAsync(b, 0, L.total, st));
+    h->phase = kWarmup;
+    h->steps = 0;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_warmup_step(onebit_adam_t h, float* x, const void* grads, float lr,
+                            void* stream) {
+    if (!valid_handle(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
+    if (h->phase != kWarmup) return ONEBIT_ERR_PHASE;
+    if (h->geo.d == 0) return ONEBIT_OK;
+    if (x == nullptr || grads == nullptr) return ONEBIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(grads)) return ONEBIT_ERR_ALIGN;
+    cudaStream_t st = as_stream(stream);
+    return h->gtype == ONEBIT_BF16 ? launch_warmup<uint16_t>(h, x, grads, lr, st)
+                                   : launch_warmup<float>(h, x, grads, lr, st);
+}
+
+int onebit_adam_freeze_variance(onebit_adam_t h, void* stream) {
+    if (!valid_handle(h)) return ONEBIT_ERR_ARG;
+    if (h->phase != kWarmup) return ONEBIT_ERR_PHASE;
+    cudaStream_t st = as_stream(stream);
+    const Layout& L = h->lay;
+    // residuals (lazy form: stored 0 with scale 0 rebuilds e = 0), planes, scales, partials
+    ONEBIT_CUDA(cudaMemsetAsync(h->ws + L.es, 0, L.total - L.es, st));
+    h->phase = kCompressed;
+    h->steps = 0;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, float lr,
+                                void* stream) {
+    if (!valid_handle(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (h->geo.d == 0) {
+        ++h->steps;
+        return ONEBIT_OK;
+    }
+    if (x == nullptr || grads == nullptr) return ONEBIT_ERR_ARG;
+    if (!aligned16(x) || !aligned16(grads)) return ONEBIT_ERR_ALIGN;
+    cudaStream_t st = as_stream(stream);
+    const Geometry& g = h->geo;
+    const unsigned blocks = (unsigned)step_blocks(g);
+    int rc;
+
+    record(h, 0, st);
+    rc = h->gtype == ONEBIT_BF16 ? launch_worker<uint16_t>(h, grads, st)
+                                 : launch_worker<float>(h, grads, st);
+    if (rc != ONEBIT_OK) return rc;
+    record(h, 1, st);
+    rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, h->s_out, h->s_lazy, st);
+    if (rc != ONEBIT_OK) return rc;
+    record(h, 2, st);
+    ServerArgs sa{g, h->bits_w, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s, h->status};
+    k_server<<<blocks, kThreads, (size_t)(g.W + kWarps) * sizeof(double), st>>>(sa);
+    ONEBIT_CUDA(cudaGetLastError());
+    record(h, 3, st);
+    rc = launch_scales(g, h->part_s, g.nch, h->S_out, h->S_lazy, st);
+    if (rc != ONEBIT_OK) return rc;
+    record(h, 4, st);
+    ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, h->m, x};
+    k_apply<<<blocks, kThreads, 0, st>>>(pa);
+    ONEBIT_CUDA(cudaGetLastError());
+    record(h, 5, st);
+    if (h->tcount < h->tmax) ++h->tcount;
+    ++h->steps;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_compressed_step_host(onebit_adam_t h, float* x_dev, void* grads_dev,
+                                     const void* grads_host, float* x_host, float lr,
+                                     void* stream) {
+    if (!valid_handle(h)) return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (h->geo.d == 0) return onebit_adam_compressed_step(h, x_dev, grads_dev, lr, stream);
+    if (grads_host == nullptr || x_host == nullptr || grads_dev == nullptr || x_dev == nullptr)
+        return ONEBIT_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    const uint64_t gbytes = (uint64_t)h->geo.W * h->geo.d * grad_elem_bytes(h->gtype);
+    ONEBIT_CUDA(cudaMemcpyAsync(grads_dev, grads_host, gbytes, cudaMemcpyHostToDevice, st));
+    const int rc = onebit_adam_compressed_step(h, x_dev, grads_dev, lr, stream);
+    if (rc != ONEBIT_OK) return rc;
+    ONEBIT_CUDA(cudaMemcpyAsync(x_host, x_dev, (uint64_t)h->geo.d * sizeof(float),
+                                cudaMemcpyDeviceToHost, st));
+    return ONEBIT_OK;
+}
+
+int onebit_adam_state_bytes(onebit_adam_t h, int32_t which, uint64_t* bytes) {
+    if (!valid_handle(h) || bytes == nullptr) return ONEBIT_ERR_ARG;
+    const Geometry& g = h->geo;
+    const uint64_t f = sizeof(float);
+    switch (which) {
+        case ONEBIT_STATE_M:
+        case ONEBIT_STATE_V:
+        case ONEBIT_STATE_ES: *bytes = g.d * f; break;
+        case ONEBIT_STATE_EW: *bytes = (uint64_t)g.W * g.d * f; break;
+        case ONEBIT_STATE_SW: *bytes = (uint64_t)g.W * g.nch * f; break;
+        case ONEBIT_STATE_SS: *bytes = g.nch * f; break;
+        case ONEBIT_STATE_BITSW: *bytes = (uint64_t)g.W * h->nw * sizeof(uint32_t); break;
+        case ONEBIT_STATE_BITSS: *bytes = h->nw * sizeof(uint32_t); break;
+        default: return ONEBIT_ERR_ARG;
+    }
+    return ONEBIT_OK;
+}
+
+int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* stream) {
+    uint64_t bytes = 0;
+    int rc = onebit_adam_state_bytes(h, which, &bytes);
+    if (rc != ONEBIT_OK) return rc;
+    if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
+    if (bytes == 0) return ONEBIT_OK;
+    if (dst == nullptr) return ONEBIT_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    const Geometry& g = h->geo;
+    const auto D2D = cudaMemcpyDeviceToDevice;
+    switch (which) {
+        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m, bytes, D2D, st)); break;
+        case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->v, bytes, D2D, st)); break;
+        case ONEBIT_STATE_SW: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->s_out, bytes, D2D, st)); break;
+        case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out, bytes, D2D, st)); break;
+        case ONEBIT_STATE_BITSW:
+            ONEBIT_CUDA(cudaMemcpy2DAsync(dst, h->nw * sizeof(uint32_t), h->bits_w,
+                                          g.ldw * sizeof(uint32_t), h->nw * sizeof(uint32_t),
+                                          g.W, D2D, st));
+            break;
+        case ONEBIT_STATE_BITSS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->bits_s, bytes, D2D, st)); break;
+        case ONEBIT_STATE_EW:
+        case ONEBIT_STATE_ES: {
+            const bool wk = which == ONEBIT_STATE_EW;
+            const int rc2 = launch_materialize(h, wk, 0, g.d, static_cast<float*>(dst), st);
+            if (rc2 != ONEBIT_OK) return rc2;
+            break;
+        }
+        default: return ONEBIT_ERR_ARG;
+    }
+    return ONEBIT_OK;
+}
+
+int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void* dst,
+                                void* stream) {
+    if (!valid_handle(h)) return ONEBIT_ERR_ARG;
+    if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
+    const Geometry& g = h->geo;
+    if (k < 0 || k >= g.nch || dst == nullptr) return ONEBIT_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    const int64_t i0 = k * g.C, n = std::min(g.C, g.d - i0);
+    const int64_t w0 = i0 / 32, nwk = ceil_div(n, 32);
+    const uint64_t f = sizeof(float), u = sizeof(uint32_t);
+    const auto D2D = cudaMemcpyDeviceToDevice;
+    switch (which) {
+        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m + i0, n * f, D2D, st)); break;
+        case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->v + i0, n * f, D2D, st)); break;
+        case ONEBIT_STATE_EW:
+        case ONEBIT_STATE_ES:
+            return launch_materialize(h, which == ONEBIT_STATE_EW, i0, n,
+                                      static_cast<float*>(dst), st);
+        case ONEBIT_STATE_SW:
+            ONEBIT_CUDA(cudaMemcpy2DAsync(dst, f, h->s_out + k, g.nch * f, f, g.W, D2D, st));
+            break;
+        case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out + k, f, D2D, st)); break;
+        case ONEBIT_STATE_BITSW:
+            ONEBIT_CUDA(cudaMemcpy2DAsync(dst, nwk * u, h->bits_w + w0, g.ldw * u, nwk * u, g.W,
+                                          D2D, st));
+            break;
+        case ONEBIT_STATE_BITSS:
+            ONEBIT_CUDA(cudaMemcpyAsync(dst, h->bits_s + w0, nwk * u, D2D, st));
+            break;
+        default: return ONEBIT_ERR_ARG;
+    }
+    return ONEBIT_OK;
+}
+
+int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void* stream) {
+    uint64_t bytes = 0;
+    int rc = onebit_adam_state_bytes(h, which, &bytes);
+    if (rc != ONEBIT_OK) return rc;
+    if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
+    if (which != ONEBIT_STATE_M && which != ONEBIT_STATE_V && which != ONEBIT_STATE_EW &&
+        which != ONEBIT_STATE_ES)
+        return ONEBIT_ERR_ARG;
+    if (bytes == 0) return ONEBIT_OK;
+    if (src == nullptr) return ONEBIT_ERR_ARG;
+    cudaStream_t st = as_stream(stream);
+    const Geometry& g = h->geo;
+    const auto D2D = cudaMemcpyDeviceToDevice;
+    const uint64_t f = sizeof(float);
+    switch (which) {
+        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(h->m, src, bytes, D2D, st)); break;
+        case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(h->v, src, bytes, D2D, st)); break;
+        case ONEBIT_STATE_EW:
+            // explicit residual with a zero rebuild scale: e = stored - (+-0) = stored exactly
+            ONEBIT_CUDA(cudaMemcpy2DAsync(h->ew, g.ld * f, src, g.d * f, g.d * f, g.W, D2D, st));
+            ONEBIT_CUDA(cudaMemsetAsync(h->s_lazy, 0, (uint64_t)g.W * g.nch * f, st));
+            ONEBIT_CUDA(cudaMemsetAsync(h->s_out, 0, (uint64_t)g.W * g.nch * f, st));
+            break;
+        case ONEBIT_STATE_ES:
+            ONEBIT_CUDA(cudaMemcpyAsync(h->es, src, bytes, D2D, st));
+            ONEBIT_CUDA(cudaMemsetAsync(h->S_lazy, 0, g.nch * f, st));
+            ONEBIT_CUDA(cudaMemsetAsync(h->S_out, 0, g.nch * f, st));
+            break;
+        default: return ONEBIT_ERR_ARG;
+    }
+    return ONEBIT_OK;
+}
+
+int onebit_adam_status(onebit_adam_t h, void* stream, uint32_t* flags) {
+    if (!valid_handle(h) || flags == nullptr) return ONEBIT_ERR_ARG;
+    *flags = 0;
+    if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
+    cudaStream_t st = as_stream(stream);
+    uint32_t hostv = 0;
+    ONEBIT_CUDA(cudaMemcpyAsync(&hostv, h->status, sizeof hostv, cudaMemcpyDeviceToHost, st));
+    ONEBIT_CUDA(cudaMemsetAsync(h->status, 0, sizeof hostv, st));
+    ONEBIT_CUDA(cudaStreamSynchronize(st));
+    *flags = hostv;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_info(onebit_adam_t h, int64_t out[8]) {
+    if (!valid_handle(h) || out == nullptr) return ONEBIT_ERR_ARG;
+    out[0] = h->geo.d;
+    out[1] = h->geo.W;
+    out[2] = h->geo.C;
+    out[3] = h->geo.nch;
+    out[4] = h->phase;
+    out[5] = h->steps;
+    out[6] = h->gtype;
+    out[7] = kLaunchesPerStep;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_timing(onebit_adam_t h, int32_t max_steps) {
+    if (!valid_handle(h) || max_steps < 0 || max_steps > (1 << 20)) return ONEBIT_ERR_ARG;
+    free_events(h);
+    if (max_steps == 0) return ONEBIT_OK;
+    h->ev.resize((size_t)max_steps * kEventsPerStep, nullptr);
+    for (auto& e : h->ev) {
+        const cudaError_t rc = cudaEventCreate(&e);
+        if (rc != cudaSuccess) {
+            e = nullptr;
+            for (auto& f : h->ev)
+                if (f) cudaEventDestroy(f);
+            h->ev.clear();
+            return cuda_fail(rc);
+        }
+    }
+    h->tmax = max_steps;
+    h->tcount = 0;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps) {
+    if (!valid_handle(h) || ms_out == nullptr || steps == nullptr) return ONEBIT_ERR_ARG;
+    for (int i = 0; i < kLaunchesPerStep; ++i) ms_out[i] = 0.0;
+    *steps = h->tcount;
+    if (h->tcount == 0) return ONEBIT_OK;
+    ONEBIT_CUDA(cudaEventSynchronize(h->ev[(size_t)h->tcount * kEventsPerStep - 1]));
+    for (int32_t s = 0; s < h->tcount; ++s) {
+        for (int i = 0; i < kLaunchesPerStep; ++i) {
+            float ms = 0.0f;
+            ONEBIT_CUDA(cudaEventElapsedTime(&ms, h->ev[(size_t)s * kEventsPerStep + i],
+                                             h->ev[(size_t)s * kEventsPerStep + i + 1]));
+            ms_out[i] += ms;
+        }
+    }
+    h->tcount = 0;
+    return ONEBIT_OK;
+}
+
+void onebit_adam_destroy(onebit_adam_t h) {
+    if (h == nullptr) return;
+    free_events(h);
+    delete h;
+}
+
+int onebit_pack(const float* x, int64_t n, uint32_t* words, void* stream) {
+    if (n < 0) return ONEBIT_ERR_ARG;
+    if (n == 0) return ONEBIT_OK;
+    if (x == nullptr || words == nullptr) return ONEBIT_ERR_ARG;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(words) & 3u)) return ONEBIT_ERR_ALIGN;
+    if (n > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
+    k_pack<<<(unsigned)ceil_div(n, kSeg), kThreads, 0, as_stream(stream)>>>(x, n, words);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t C, float* out,
+                  void* stream) {
+    if (n < 0 || C < 1) return ONEBIT_ERR_ARG;
+    if (n == 0) return ONEBIT_OK;
+    if (words == nullptr || scales == nullptr || out == nullptr) return ONEBIT_ERR_ARG;
+    if (!aligned16(out) || (reinterpret_cast<uintptr_t>(words) & 3u) ||
+        (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return ONEBIT_ERR_ALIGN;
+    if (n > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
+    k_unpack<<<(unsigned)ceil_div(n, kSeg), kThreads, 0, as_stream(stream)>>>(words, scales, n,
+                                                                            C, out);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+}  // extern "C"

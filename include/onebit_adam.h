@@ -1,0 +1,214 @@
+/*
+ * onebit_adam.h -- C ABI of the B200 (sm_100a) library for the data-parallel hot path of the
+ * compression phase of 1-bit Adam (Tang et al., arXiv 2102.02888).
+ *
+ * The method (as the pages describe it):
+ *   - "1-bit Adam" index page (mlsanity.com/paper/2102.02888), Abstract: Adam's variance becomes
+ *     stable after a warm-up phase and is then used as a fixed preconditioner for the rest of
+ *     training (the compression phase), where communication uses error-compensated 1-bit
+ *     compression.
+ *   - LIT-278 note (dmarx.github.io anthology), Key takeaways: the compression phase is 1-bit
+ *     compressed momentum SGD with that fixed preconditioner; Theorem 1 assumes
+ *     error-compensated 1-bit compression with per-chunk scaling.
+ *   - LIT-278 note, "What the evidence does not cover": the warm-up is full-precision Adam; the
+ *     compressed allreduce is a custom collective.
+ *
+ * In this library the W data-parallel workers are a batch dimension in one GPU's memory: the
+ * compressed allreduce is a gather over the W workers' packed sign planes in device memory.
+ *
+ * Conventions (all calls):
+ *   - Every pointer named *_dev or documented as device memory is a CUDA device pointer owned
+ *     by the caller, 16-byte aligned, and must stay valid until the work queued on the stream
+ *     has finished. The library never allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device work
+ *     is queued on it asynchronously; argument errors are detected on the host and returned
+ *     before anything is queued.
+ *   - Return values: ONEBIT_OK (0) or a negative onebit_status. ONEBIT_ERR_CUDA means a CUDA
+ *     runtime call or kernel launch failed (the CUDA error string is kept, see onebit_last_error).
+ *   - Floating point: every fp32 operation of the method is one IEEE round-to-nearest-even
+ *     operation (no fused multiply-add, no flush-to-zero); norms and the server average are
+ *     accumulated in fp64.
+ *   - Sign convention: bit = (x >= 0) (so +0 and -0 give 1, NaN gives 0). Packed planes are
+ *     LSB-first uint32 words: element i is bit i%32 of word i/32; bits past the end are 0.
+ *   - Chunks: contiguous runs of C elements of the flat d-vector, the last one possibly shorter;
+ *     each chunk has its own fp32 scale = sqrt(sum of squares / chunk length).
+ */
+#ifndef ONEBIT_ADAM_H
+#define ONEBIT_ADAM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct onebit_adam_s* onebit_adam_t; /* opaque, host-owned handle */
+
+typedef enum {
+    ONEBIT_OK = 0,
+    ONEBIT_ERR_ARG = -1,     /* bad size, null pointer, unknown enum value */
+    ONEBIT_ERR_ALIGN = -2,   /* C not a multiple of 32, pointer not 16-byte aligned */
+    ONEBIT_ERR_PHASE = -3,   /* warm-up after the freeze, compressed step before it, unbound */
+    ONEBIT_ERR_CUDA = -4,    /* a CUDA call failed */
+    ONEBIT_ERR_SPACE = -5    /* workspace smaller than onebit_adam_workspace_bytes */
+} onebit_status;
+
+typedef enum { ONEBIT_F32 = 0, ONEBIT_BF16 = 1 } onebit_dtype;
+
+/* State selectors for onebit_adam_get_state / onebit_adam_set_state. */
+typedef enum {
+    ONEBIT_STATE_M = 0,     /* momentum m, fp32[d]                                   (get/set) */
+    ONEBIT_STATE_V = 1,     /* variance v (frozen after the freeze), fp32[d]         (get/set) */
+    ONEBIT_STATE_EW = 2,    /* worker residuals e_w, fp32[W][d]                      (get/set) */
+    ONEBIT_STATE_ES = 3,    /* server residual e_s, fp32[d]                          (get/set) */
+    ONEBIT_STATE_SW = 4,    /* last step's worker scales s, fp32[W][nch]             (get) */
+    ONEBIT_STATE_SS = 5,    /* last step's server scales S, fp32[nch]                (get) */
+    ONEBIT_STATE_BITSW = 6, /* last step's worker sign planes, uint32[W][ceil(d/32)] (get) */
+    ONEBIT_STATE_BITSS = 7  /* last step's server sign plane, uint32[ceil(d/32)]     (get) */
+} onebit_state;
+
+/* Device status flags (onebit_adam_status). */
+#define ONEBIT_FLAG_NAN_WORKER 1u /* some worker's x_w was NaN (its bit is 0) */
+#define ONEBIT_FLAG_NAN_SERVER 2u /* some server z was NaN */
+
+/*
+ * Create a handle for d parameters, W workers, chunk length C ("1-bit Adam" index page,
+ * Abstract; LIT-278 note, Key takeaways: per-chunk scaling). Host only, no device work.
+ *   d >= 0 (d = 0 makes every step a no-op), 1 <= W <= 256, C >= 32 and C % 32 == 0
+ *   (ONEBIT_ERR_ALIGN otherwise; C need not divide d), 0 <= beta1, beta2 < 1, eps >= 0, all
+ *   finite. *out receives the handle; release it with onebit_adam_destroy.
+ */
+int onebit_adam_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                     float beta2, float eps);
+
+/* Bytes of device workspace the handle needs for gradients of type grad_dtype. */
+int onebit_adam_workspace_bytes(onebit_adam_t h, int32_t grad_dtype, uint64_t* bytes);
+
+/*
+ * Give the handle its device workspace (caller-owned, 256-byte aligned, at least
+ * onebit_adam_workspace_bytes long) and fix the gradient type. Zeroes m and v on `stream`
+ * (Adam's initial state) and puts the handle in the warm-up phase. The workspace holds m, v,
+ * the residuals, the sign planes, the scales and the fp64 norm partials.
+ */
+int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t grad_dtype,
+                     void* stream);
+
+/*
+ * One full-precision Adam warm-up step (LIT-278 note, "What the evidence does not cover": the
+ * warm-up runs uncompressed Adam). grads: [W][d] of the bound type, device; x: fp32[d], device,
+ * updated in place. gbar = fp64 average over workers rounded once; m = b1 m + (1-b1) gbar;
+ * v = b2 v + (1-b2) gbar^2; x -= lr * (m / (sqrt(v) + eps)); no bias correction.
+ * ONEBIT_ERR_PHASE after onebit_adam_freeze_variance.
+ */
+int onebit_adam_warmup_step(onebit_adam_t h, float* x, const void* grads, float lr,
+                            void* stream);
+
+/*
+ * End the warm-up: v becomes the fixed preconditioner ("1-bit Adam" index page, Abstract;
+ * LIT-278 note, tag list: freeze the variance before compressing). Worker and server residuals
+ * and all scales start at zero. Allowed once; ONEBIT_ERR_PHASE afterwards.
+ */
+int onebit_adam_freeze_variance(onebit_adam_t h, void* stream);
+
+/*
+ * One compressed step (LIT-278 note, Key takeaways: 1-bit compressed momentum SGD with error
+ * feedback, per-chunk scaling, frozen-variance preconditioner). grads: [W][d], device; x:
+ * fp32[d], device, updated in place. For each worker w and element i:
+ *   x_w = (b1 m + (1-b1) g_w) + e_w;  s_w,k = ||x_w[chunk k]||_2 / sqrt(C_k);
+ *   e_w = x_w - (x_w >= 0 ? s_w,k : -s_w,k)
+ * then the compressed allreduce over the W packed planes, per element of chunk k:
+ *   z = fl32(fp64 sum_w (+-s_w,k) / W) + e_s;  S_k = ||z[chunk k]||_2 / sqrt(C_k);
+ *   e_s = z - (z >= 0 ? S_k : -S_k)
+ * and every worker's apply: m = (z >= 0 ? S_k : -S_k); x -= lr * (m / (sqrt(v) + eps)).
+ * ONEBIT_ERR_PHASE before onebit_adam_freeze_variance.
+ */
+int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, float lr,
+                                void* stream);
+
+/*
+ * The same compressed step fed from host memory: copies grads_host ([W][d] of the bound type,
+ * pinned host memory for an asynchronous copy) into grads_dev, runs the step on x_dev, and
+ * copies the updated x_dev back into x_host (fp32[d]). All copies and kernels are queued on
+ * `stream`; the host buffers must not be touched until the stream has finished.
+ */
+int onebit_adam_compressed_step_host(onebit_adam_t h, float* x_dev, void* grads_dev,
+                                     const void* grads_host, float* x_host, float lr,
+                                     void* stream);
+
+/*
+ * Copy one piece of state into dst (device memory, contiguous, the size listed in
+ * onebit_state; onebit_adam_state_bytes gives it). Residuals come back explicit.
+ */
+int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* stream);
+
+/*
+ * Copy the part of one piece of state that belongs to chunk k (0 <= k < number of chunks) into
+ * dst (device memory, contiguous): M, V, ES: fp32[C_k]; EW: fp32[W][C_k]; SW: fp32[W];
+ * SS: fp32[1]; BITSW: uint32[W][ceil(C_k/32)]; BITSS: uint32[ceil(C_k/32)]. Chunks are
+ * independent, so a sample of chunks checks every output that depends on them without
+ * copying whole W x d buffers. Residuals come back explicit.
+ */
+int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void* dst,
+                                void* stream);
+
+/*
+ * Overwrite one piece of state (M, V, EW or ES) from src (device memory, contiguous). Used to
+ * resume from a checkpoint: a fresh handle that is bound, frozen and given M, V, EW and ES of
+ * another handle continues bit-identically. Setting EW or ES clears the reported scales of the
+ * last step. ONEBIT_ERR_ARG for the read-only selectors.
+ */
+int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void* stream);
+
+/* Size in bytes of one piece of state. */
+int onebit_adam_state_bytes(onebit_adam_t h, int32_t which, uint64_t* bytes);
+
+/*
+ * Wait for `stream`, then return the device status flags (ONEBIT_FLAG_*) gathered since the
+ * last call in *flags and clear them.
+ */
+int onebit_adam_status(onebit_adam_t h, void* stream, uint32_t* flags);
+
+/*
+ * Shape and progress: out[0..7] = d, W, C, number of chunks, phase (0 unbound, 1 warm-up,
+ * 2 compressed), compressed steps taken, gradient dtype (-1 unbound), kernel launches per
+ * compressed step.
+ */
+int onebit_adam_info(onebit_adam_t h, int64_t out[8]);
+
+/*
+ * Per-kernel timing with CUDA events recorded on the launching stream. max_steps > 0 starts
+ * recording the next max_steps compressed steps (later steps are not recorded); 0 stops and
+ * frees the events. onebit_adam_timing_read waits for the last recorded event and returns, in
+ * ms_out[0..4], the summed device time of the worker kernel, the worker-scale reduction, the
+ * server kernel, the server-scale reduction and the apply kernel, and the number of recorded
+ * steps in *steps; it then starts a new recording window of the same length.
+ */
+int onebit_adam_timing(onebit_adam_t h, int32_t max_steps);
+int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps);
+
+/* Release the handle (not the workspace, which the caller owns). NULL is ignored. */
+void onebit_adam_destroy(onebit_adam_t h);
+
+/*
+ * Sign-pack n fp32 values (device) into ceil(n/32) LSB-first words (device): bit = x >= 0;
+ * padding bits are 0. The 1-bit message of the method without its scale. n >= 0.
+ */
+int onebit_pack(const float* x, int64_t n, uint32_t* words, void* stream);
+
+/*
+ * Decompress: out[i] = bit_i ? scales[i / C] : -scales[i / C] for i < n (all device). C >= 1.
+ */
+int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t C, float* out,
+                  void* stream);
+
+/* Static description of a status code. */
+const char* onebit_strerror(int32_t code);
+
+/* Text of the last CUDA error this thread saw in the library ("" if none). */
+const char* onebit_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ONEBIT_ADAM_H */

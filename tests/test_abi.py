@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every function the public header
+declares, and rejects bad arguments on the host before any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import communication_compressed_optimizer_momentum_b200 as ob
+from communication_compressed_optimizer_momentum_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "onebit_adam.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(onebit_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from communication_compressed_optimizer_momentum_b200 import build
+    build.build()
+    return _abi.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("onebit_adam_init", "onebit_adam_warmup_step", "onebit_adam_freeze_variance",
+              "onebit_adam_compressed_step", "onebit_pack", "onebit_unpack"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    # the binding wraps each of them with the same name
+    assert set(names) <= set(_abi.SIGNATURES)
+    for n in names:
+        assert hasattr(ob, n), n
+
+
+def test_init_validates_arguments(lib):
+    h = ctypes.c_void_p()
+    ok = lib.onebit_adam_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8)
+    assert ok == 0 and h.value
+    lib.onebit_adam_destroy(h)
+    bad = [
+        ((-1, 4, 256, 0.9, 0.999, 1e-8), -1),     # negative d
+        ((1000, 0, 256, 0.9, 0.999, 1e-8), -1),   # no workers
+        ((1000, 257, 256, 0.9, 0.999, 1e-8), -1), # too many workers
+        ((1000, 4, 0, 0.9, 0.999, 1e-8), -1),     # empty chunk
+        ((1000, 4, 100, 0.9, 0.999, 1e-8), -2),   # chunk not a multiple of 32
+        ((1000, 4, 256, 1.0, 0.999, 1e-8), -1),   # beta1 out of [0, 1)
+        ((1000, 4, 256, 0.9, -0.1, 1e-8), -1),    # beta2 out of [0, 1)
+        ((1000, 4, 256, 0.9, 0.999, -1.0), -1),   # negative eps
+        ((1000, 4, 256, float("nan"), 0.999, 1e-8), -1),
+    ]
+    for args, code in bad:
+        h = ctypes.c_void_p()
+        assert lib.onebit_adam_init(ctypes.byref(h), *args) == code, args
+        assert not h.value
+    assert lib.onebit_adam_init(None, 10, 1, 32, 0.9, 0.999, 1e-8) == -1
+
+
+def test_empty_vector_is_a_valid_problem(lib):
+    h = ob.onebit_adam_init(0, 3, 64)
+    info = ob.onebit_adam_info(h)
+    assert info["d"] == 0 and info["nch"] == 0 and info["phase"] == 0
+    assert ob.onebit_adam_state_bytes(h, ob.STATE["e_w"]) == 0
+    ob.onebit_adam_destroy(h)
+
+
+def test_phase_rules_before_bind(lib):
+    """Unbound handles refuse every step with ONEBIT_ERR_PHASE, before touching the device."""
+    h = ob.onebit_adam_init(4096, 2, 1024)
+    for fn in (lambda: lib.onebit_adam_compressed_step(h, None, None, ctypes.c_float(1e-3), None),
+               lambda: lib.onebit_adam_warmup_step(h, None, None, ctypes.c_float(1e-3), None),
+               lambda: lib.onebit_adam_freeze_variance(h, None)):
+        assert fn() == -3
+    flags = ctypes.c_uint32()
+    assert lib.onebit_adam_status(h, None, ctypes.byref(flags)) == -3
+    ob.onebit_adam_destroy(h)
+
+
+def test_workspace_size_and_bind_checks(lib):
+    h = ob.onebit_adam_init(100_003, 5, 4096)
+    n32 = ob.onebit_adam_workspace_bytes(h, ob.ONEBIT_F32)
+    # m, v, e_s, e_w (W+3 fp32 vectors) plus planes, scales and partials
+    assert n32 >= (5 + 3) * 100_003 * 4
+    with pytest.raises(ob.OneBitError):
+        ob.onebit_adam_workspace_bytes(h, 7)
+    # misaligned or short workspaces are rejected on the host
+    assert lib.onebit_adam_bind(h, ctypes.c_void_p(0x1001), n32, 0, None) == -2
+    assert lib.onebit_adam_bind(h, ctypes.c_void_p(0x100000), n32 - 1, 0, None) == -5
+    assert lib.onebit_adam_bind(h, ctypes.c_void_p(0x100000), n32, 3, None) == -1
+    assert lib.onebit_adam_bind(h, None, n32, 0, None) == -1
+    ob.onebit_adam_destroy(h)
+
+
+def test_state_sizes(lib):
+    d, W, C = 1000, 3, 256
+    h = ob.onebit_adam_init(d, W, C)
+    nch, nw = 4, 32
+    exp = {"m": d * 4, "v": d * 4, "e_w": W * d * 4, "e_s": d * 4, "s": W * nch * 4,
+           "S": nch * 4, "bits_w": W * nw * 4, "bits_s": nw * 4}
+    for k, v in exp.items():
+        assert ob.onebit_adam_state_bytes(h, ob.STATE[k]) == v, k
+    with pytest.raises(ob.OneBitError):
+        ob.onebit_adam_state_bytes(h, 99)
+    ob.onebit_adam_destroy(h)
+
+
+def test_pack_unpack_host_checks(lib):
+    assert lib.onebit_pack(None, -1, None, None) == -1
+    assert lib.onebit_pack(None, 0, None, None) == 0          # empty input: nothing to do
+    assert lib.onebit_pack(ctypes.c_void_p(0x1004), 10, ctypes.c_void_p(0x2000), None) == -2
+    assert lib.onebit_unpack(None, None, 0, 32, None, None) == 0
+    assert lib.onebit_unpack(None, None, 10, 0, None, None) == -1
+
+
+def test_timing_arguments(lib):
+    h = ob.onebit_adam_init(1000, 2, 256)
+    with pytest.raises(ob.OneBitError):
+        ob.onebit_adam_timing(h, -1)
+    ob.onebit_adam_timing(h, 0)
+    ms, n = ob.onebit_adam_timing_read(h)
+    assert n == 0 and all(v == 0.0 for v in ms.values())
+    ob.onebit_adam_destroy(h)
+
+
+def test_strerror_covers_codes(lib):
+    for c in (0, -1, -2, -3, -4, -5):
+        assert lib.onebit_strerror(c).decode() != "unknown status"
+    assert lib.onebit_strerror(12345).decode() == "unknown status"
