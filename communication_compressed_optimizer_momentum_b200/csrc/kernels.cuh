@@ -2,10 +2,13 @@
 //
 // Every kernel here streams HBM: there is no dense contraction in the method, so the tensor
 // cores play no part and the design goal is bytes moved once, coalesced, with enough loads in
-// flight. The work unit is a SEGMENT: kSeg = 4096 consecutive elements that never cross a chunk
-// boundary (chunk k = elements [kC, kC + C_k), LIT-278 note, Key takeaways: per-chunk scaling).
-// A block owns one segment; thread t owns kItems groups of kVec = 4 consecutive elements at
-// offsets (it * kThreads + t) * 4, so each warp-wide access is one contiguous 512-byte run.
+// flight. The work unit is a SEGMENT of consecutive elements that never crosses a chunk
+// boundary (chunk k = elements [kC, kC + C_k), LIT-278 note, Key takeaways: per-chunk scaling):
+// kSeg = 2048 elements for the worker, apply and warm-up kernels, kSegS = 4096 for the server
+// kernel. A block owns one segment; in the 2048-element kernels thread t owns kItems groups of
+// kVec = 4 consecutive elements at offsets (it * kThreads + t) * 4, so each warp-wide access is
+// one contiguous 512-byte run. Small per-thread state (about 40 registers) keeps 48 warps per SM
+// in flight, which is what hides HBM latency here.
 //
 // Determinism: chunk norms are fp64 sums in a fixed tree (thread -> warp butterfly -> block in
 // warp order -> segments in order), so a run is bit-reproducible; no float atomics anywhere.
@@ -24,18 +27,24 @@ namespace onebit {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kVec = 4;
-constexpr int kItems = 4;
-constexpr int kSeg = kThreads * kVec * kItems;  // 4096 elements per segment
+constexpr int kItems = 2;
+constexpr int kSeg = kThreads * kVec * kItems;  // 2048 elements per segment
+constexpr int kSrvVec = 8;                      // server kernel: elements per thread per item
+constexpr int kSrvItems = 2;
+constexpr int kSegS = kThreads * kSrvVec * kSrvItems;  // 4096 elements per server segment
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kNanWorker = 1u;
 constexpr uint32_t kNanServer = 2u;
+constexpr uint32_t kWaitTimeout = 4u;           // a bounded wait gave up (see k_server)
+constexpr int kSpinLimit = 1 << 22;
 
 // Shape of the problem and of the library's own buffers.
 struct Geometry {
     int64_t d;     // parameters
     int64_t C;     // chunk length (multiple of 32)
     int64_t nch;   // chunks, ceil(d / C)
-    int64_t nseg;  // segments per full chunk, ceil(C / kSeg)
+    int64_t nseg;    // kSeg segments per full chunk
+    int64_t nseg_s;  // kSegS segments per full chunk
     int64_t ld;    // row length (elements) of the library's fp32 [W][ld] residual buffer
     int64_t ldw;   // row length (words) of a packed sign plane
     int32_t W;     // workers
@@ -51,17 +60,19 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
-// Segment of this block: chunk k, segment j within it, global start `base`, length `len`.
-__device__ __forceinline__ bool block_segment(const Geometry& g, int64_t& k, int64_t& j,
-                                              int64_t& base, int64_t& len) {
-    k = (int64_t)blockIdx.x / g.nseg;
-    j = (int64_t)blockIdx.x - k * g.nseg;
+// Segment of this block (SEG elements, nseg of them per full chunk): chunk k, segment j within
+// it, global start `base`, length `len`.
+template <int SEG>
+__device__ __forceinline__ bool block_segment(const Geometry& g, int64_t nseg, int64_t& k,
+                                              int64_t& j, int64_t& base, int64_t& len) {
+    k = (int64_t)blockIdx.x / nseg;
+    j = (int64_t)blockIdx.x - k * nseg;
     const int64_t c0 = k * g.C;
     const int64_t clen = min(g.C, g.d - c0);
-    const int64_t s0 = j * kSeg;
+    const int64_t s0 = j * SEG;
     if (s0 >= clen) return false;
     base = c0 + s0;
-    len = min((int64_t)kSeg, clen - s0);
+    len = min((int64_t)SEG, clen - s0);
     return true;
 }
 
@@ -156,11 +167,13 @@ struct WorkerArgs {
     uint32_t* status;
 };
 
+// 8 resident blocks per SM (at most 32 registers a thread): the kernel is latency-bound on HBM
+// and more warps in flight beat deeper per-thread prefetch (measured on B200).
 template <typename GT, bool VEC>
-__global__ void __launch_bounds__(kThreads) k_worker(const WorkerArgs a) {
+__global__ void __launch_bounds__(kThreads, 8) k_worker(const WorkerArgs a) {
     extern __shared__ double red_w[];  // [W][kWarps]
     int64_t k, j, base, len;
-    if (!block_segment(a.geo, k, j, base, len)) return;
+    if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = a.geo.W;
 
@@ -223,8 +236,9 @@ __global__ void __launch_bounds__(kThreads) k_worker(const WorkerArgs a) {
 
 template <int TPR>
 __global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t rows,
-                                                     int64_t nch, int64_t nseg, int64_t C,
-                                                     int64_t d, float* out, float* lazy) {
+                                                     int64_t nch, int64_t nseg, int64_t seg,
+                                                     int64_t C, int64_t d, float* out,
+                                                     float* lazy) {
     __shared__ double red[kWarps];
     const int64_t r = (int64_t)blockIdx.x * (kThreads / TPR) + threadIdx.x / TPR;
     const int sub = threadIdx.x % TPR;
@@ -234,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t
     if (active) {
         const int64_t k = r % nch;
         clen = min(C, d - k * C);
-        const int64_t nsk = (clen + kSeg - 1) / kSeg;
+        const int64_t nsk = (clen + seg - 1) / seg;
         const double* p = part + r * nseg;
         for (int64_t jj = sub; jj < nsk; jj += TPR) acc += p[jj];
     }
@@ -252,10 +266,79 @@ __global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t
 }
 
 // ------------------------------------------------------------------------------------------
-// K2: the server side of the compressed allreduce for one segment of chunk k.
-//   y = fl32(fp64 sum_w (+-s_w,k) / W) with the workers taken in order 0..W-1;
-//   z = y + e_s;  bit = z >= 0;  store z (lazy server residual);  fp64 partial of sum z^2.
+// TMA bulk copies (global -> shared, completion counted on an mbarrier) and bounded waits.
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// 1-D bulk copy; dst, src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of the barrier, giving up after kSpinLimit polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    for (int i = 0; i < kSpinLimit; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+// ------------------------------------------------------------------------------------------
+// K2: the server side of the compressed allreduce for one kSegS segment of chunk k.
+//   y = fl32(fp64 sum_w (+-s_w,k) / W);  z = y + e_s;  bit = z >= 0;
+//   store z (lazy server residual);  fp64 partial of sum z^2.
 // LIT-278 note, Key takeaways and "What the evidence does not cover" (the compressed allreduce).
+//
+// Staging. Thread 0 starts one TMA bulk copy per worker (that worker's sign words of the
+// segment, at most 512 bytes) into shared memory; while they land, the block loads the scales,
+// checks exactness and builds its lookup tables, and every thread fetches its residuals.
+//
+// Decoding. Thread t owns 8 consecutive elements: byte (t % 4) of one 32-element word of every
+// worker's plane. For each group of 8 workers it gathers their 8 bytes (__byte_perm), transposes
+// the 8x8 bit block so that byte c holds element c's 8 worker bits, and looks the 8-bit pattern
+// up in a per-block table of the sums of (+-s) over that group. Every partial sum of the W
+// values +-s_w is exact in fp64 when sum |s_w| <= 2^53 * u (u = the smallest ulp among the
+// nonzero s_w), so then the grouping cannot change the result. The block picks one of four
+// decodes, all bit-identical to the in-order fp64 sum of the definition:
+//   kModeY     W <= 8: one table of y itself (its entries are the in-order sums);
+//   kModeInt   exact and sum |s_w| / u < 2^31: the +-s_w are integers in units of u, the tables
+//              are int32 and a lookup costs one integer add; y = fl32(A * u / W);
+//   kModeF64   exact: fp64 tables;
+//   kModeSeq   otherwise (or NaN/inf scales): worker by worker in order 0..W-1.
+
+enum ServerMode : int { kModeY = 0, kModeInt = 1, kModeF64 = 2, kModeSeq = 3 };
+
+constexpr int kSegWords = kSegS / 32;      // sign words per worker per server segment
+constexpr int kTileRow = kSegWords + 4;    // staged row: the segment's words plus up to 3 words
+                                           // before them (copies start 16-byte aligned)
 
 struct ServerArgs {
     Geometry geo;
@@ -264,63 +347,281 @@ struct ServerArgs {
     float* es;               // [ld] lazy server residual: holds last step's z
     const float* S_lazy;     // [nch]
     uint32_t* bits_s;        // [ldw]
-    double* part_s;          // [nch][nseg]
+    double* part_s;          // [nch][nseg_s]
     uint32_t* status;
 };
 
+// Dynamic shared memory of k_server for W workers (bytes).
+__host__ __device__ inline size_t server_smem_bytes(int W) {
+    const int wpad = (W + 7) & ~7;
+    return 32                                                   // mbarrier, mode, unit
+         + (size_t)W * kTileRow * sizeof(uint32_t)              // staged sign words
+         + (size_t)wpad * sizeof(double)                        // scales
+         + (size_t)(wpad / 8) * 256 * sizeof(double)            // per-group tables
+         + 256 * sizeof(float)                                  // y table (W <= 8)
+         + kWarps * sizeof(double);                             // reduction
+}
+
+// byte i bit c  ->  byte c bit i, on (lo = bytes 0..3, hi = bytes 4..7): three delta swaps of
+// the row/column index bits; the first two stay inside each 32-bit half.
+__device__ __forceinline__ void transpose8x8(uint32_t& lo, uint32_t& hi) {
+    uint32_t t;
+    t = ((lo >> 7) ^ lo) & 0x00AA00AAu;  lo ^= t ^ (t << 7);
+    t = ((hi >> 7) ^ hi) & 0x00AA00AAu;  hi ^= t ^ (t << 7);
+    t = ((lo >> 14) ^ lo) & 0x0000CCCCu; lo ^= t ^ (t << 14);
+    t = ((hi >> 14) ^ hi) & 0x0000CCCCu; hi ^= t ^ (t << 14);
+    t = ((hi << 4) ^ lo) & 0xF0F0F0F0u;  lo ^= t;  hi ^= t >> 4;
+}
+
+// Byte `b` (0..3) of 8 words -> lo/hi whose byte i is word i's byte b.
+__device__ __forceinline__ void gather_bytes(const uint32_t (&w)[8], int b, uint32_t& lo,
+                                             uint32_t& hi) {
+    const uint32_t sel = (uint32_t)b | ((uint32_t)(4 + b) << 4);
+    const uint32_t p01 = __byte_perm(w[0], w[1], sel), p23 = __byte_perm(w[2], w[3], sel);
+    const uint32_t p45 = __byte_perm(w[4], w[5], sel), p67 = __byte_perm(w[6], w[7], sel);
+    lo = __byte_perm(p01, p23, 0x5410);
+    hi = __byte_perm(p45, p67, 0x5410);
+}
+
+__device__ __forceinline__ uint32_t byte_of(uint32_t lo, uint32_t hi, int c) {
+    return ((c < 4 ? lo : hi) >> (8 * (c & 3))) & 0xffu;
+}
+
+template <bool POW2>
+__device__ __forceinline__ float server_average(double acc, double dW, double invW) {
+    return __double2float_rn(POW2 ? acc * invW : __ddiv_rn(acc, dW));
+}
+
+template <bool POW2>
 __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
-    extern __shared__ double sm_s[];  // sw[W], then red[kWarps]
+    extern __shared__ __align__(16) unsigned char smem_srv[];
     int64_t k, j, base, len;
-    if (!block_segment(a.geo, k, j, base, len)) return;
+    if (!block_segment<kSegS>(a.geo, a.geo.nseg_s, k, j, base, len)) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = a.geo.W;
-    double* sw = sm_s;
-    double* red = sm_s + W;
-    for (int w = tid; w < W; w += kThreads) sw[w] = (double)a.s[(int64_t)w * a.geo.nch + k];
+    const int wpad = (W + 7) & ~7, ngroups = wpad / 8;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem_srv);
+    int* mode_p = reinterpret_cast<int*>(smem_srv + 8);
+    int* emin_p = reinterpret_cast<int*>(smem_srv + 12);    // smallest effective exponent
+    double* unit_p = reinterpret_cast<double*>(smem_srv + 16);
+    uint32_t* tile = reinterpret_cast<uint32_t*>(smem_srv + 32);         // [W][kTileRow]
+    double* sw = reinterpret_cast<double*>(tile + (size_t)W * kTileRow);
+    double* lut = sw + wpad;                                  // fp64 tables [ngroups][256]
+    int32_t* ilut = reinterpret_cast<int32_t*>(lut);          // or int32 tables, same place
+    float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
+    double* red = reinterpret_cast<double*>(ylut + 256);
+    const double dW = (double)W, invW = 1.0 / (double)W;
+    const int64_t wbase = base >> 5;
+    // Copy words [wbase & ~3, round_up(wbase + ceil(len / 32), 4)) of every plane row: both ends
+    // 16-byte aligned and inside the row (rows are padded to a multiple of 4 words).
+    const int lead = (int)(wbase & 3);
+    const uint32_t row_bytes = (uint32_t)(((lead + (len + 31) / 32 + 3) / 4) * 16);
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)W);
+        for (int w = 0; w < W; ++w)
+            bulk_load(tile + (size_t)w * kTileRow,
+                      a.bits_w + (int64_t)w * a.geo.ldw + (wbase - lead), row_bytes, bar);
+    }
+    for (int w = tid; w < wpad; w += kThreads)
+        sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
+    // residuals of this thread's elements, fetched while the copies are in flight
+    float zp[kSrvItems][kSrvVec];
+    int nvs[kSrvItems];
+#pragma unroll
+    for (int it = 0; it < kSrvItems; ++it) {
+        const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
+        const int64_t rem = len - off;
+        nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
+        if (nvs[it] > 0) {
+            float h0[4], h1[4];
+            ld4(a.es + base + off, h0);
+            ld4(a.es + base + off + 4, h1);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
+        } else {
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) zp[it][c] = 0.0f;
+        }
+    }
     __syncthreads();
+    if (warp == 0) {
+        // exactness bound over the W scales (warp-parallel, fixed reduction order)
+        double umin = 0.0, tot = 0.0;
+        int emin = 255;
+        for (int w = lane; w < W; w += 32) {
+            const float sv = (float)sw[w];
+            if (sv == 0.0f) continue;
+            const int eb = max((int)((__float_as_uint(sv) >> 23) & 0xff), 1);
+            const double ulp = ldexp(1.0, eb - 150);
+            umin = (umin == 0.0 || ulp < umin) ? ulp : umin;
+            emin = min(emin, eb);
+            tot += fabs((double)sv);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const double u2 = __shfl_xor_sync(kFull, umin, o);
+            umin = (umin == 0.0 || (u2 != 0.0 && u2 < umin)) ? u2 : umin;
+            emin = min(emin, __shfl_xor_sync(kFull, emin, o));
+            tot += __shfl_xor_sync(kFull, tot, o);
+        }
+        if (lane == 0) {
+            int mode;
+            const bool exact = tot == 0.0 || (tot / umin <= 9007199254740992.0);
+            const int p2 = __ffs(W) - 1;                       // log2 W when W is a power of 2
+            const int kexp = emin - 150 - p2;                  // y = fl32(A) * 2^kexp
+            if (W <= 8) mode = kModeY;
+            else if (!exact) mode = kModeSeq;
+            else if (tot == 0.0 || (tot / umin <= 2147483647.0 && (!POW2 || (kexp >= -126 && kexp <= 96))))
+                mode = kModeInt;
+            else mode = kModeF64;
+            *mode_p = mode;
+            *emin_p = tot == 0.0 ? 1 : emin;
+            *unit_p = tot == 0.0 ? 0x1p-149 : umin;
+        }
+    }
+    __syncthreads();
+    const int mode = *mode_p;
+    if (mode == kModeInt) {
+        // +-s_w as exact integers in units of u = 2^(emin - 150)
+        const int emin = *emin_p;
+        for (int e = tid; e < ngroups * 256; e += kThreads) {
+            const int g = e >> 8, idx = e & 255;
+            int32_t acc = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t bits = __float_as_uint((float)sw[g * 8 + i]);
+                const int eb = (int)((bits >> 23) & 0xff);
+                const uint32_t mant = (bits & 0x7fffffu) | (eb > 0 ? 0x800000u : 0u);
+                const int32_t M = bits == 0u ? 0 : (int32_t)(mant << (max(eb, 1) - emin));
+                acc += ((idx >> i) & 1) ? M : -M;
+            }
+            ilut[e] = acc;
+        }
+    } else if (mode != kModeSeq) {
+        // fp64 tables: entry idx of group g = sum over i of (bit i of idx ? s : -s), in order
+        for (int e = tid; e < ngroups * 256; e += kThreads) {
+            const int g = e >> 8, idx = e & 255;
+            double acc = 0.0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const double sv = sw[g * 8 + i];
+                acc = __dadd_rn(acc, ((idx >> i) & 1) ? sv : -sv);
+            }
+            lut[e] = acc;
+            if (g == 0) ylut[idx] = server_average<POW2>(acc, dW, invW);
+        }
+    }
+    __syncthreads();
+    if (!mbar_wait_bounded(bar, 0)) {
+        // the copies did not land in time: record it, give them one more bounded wait, leave
+        if (tid == 0) atomicOr(a.status, kWaitTimeout);
+        mbar_wait_bounded(bar, 0);
+        return;
+    }
+    const float ykscale = __int_as_float((min(max(*emin_p - 150 - (__ffs(W) - 1), -126), 127) + 127) << 23);
+    const double unit = *unit_p;
     const float Sp = a.S_lazy[k];
-    const double dW = (double)W;
-    const uint32_t* b0 = a.bits_w + (base >> 5);
-    const int sh = 4 * (lane & 7);
     double ss = 0.0;
     bool nan_seen = false;
 #pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const int q = it * kThreads + tid;
-        const int64_t off = (int64_t)q * kVec;
-        const int nv = valid_of(len, off);
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        float zp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        if (nv > 0) {
-            ld4(a.es + base + off, zp);
-            const uint32_t* bw = b0 + (q >> 3);
-            for (int w = 0; w < W; ++w) {
-                const uint32_t nib = bw[(int64_t)w * a.geo.ldw] >> sh;
-                const double s = sw[w];
+    for (int it = 0; it < kSrvItems; ++it) {
+        const int q = it * kThreads + tid;            // 8-element group index in the segment
+        const int64_t off = (int64_t)q * kSrvVec;
+        const int nv = nvs[it];
+        const int wd = q >> 2, bsel = q & 3;           // word within the segment, byte within it
+        const uint32_t* tw = tile + lead + wd;
+        float y[kSrvVec];
+        if (mode == kModeY) {
+            uint32_t wv[8];
 #pragma unroll
-                for (int c = 0; c < kVec; ++c) acc[c] = __dadd_rn(acc[c], ((nib >> c) & 1u) ? s : -s);
+            for (int i = 0; i < 8; ++i) wv[i] = (i < W && nv > 0) ? tw[i * kTileRow] : 0u;
+            uint32_t lo, hi;
+            gather_bytes(wv, bsel, lo, hi);
+            transpose8x8(lo, hi);
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) y[c] = ylut[byte_of(lo, hi, c)];
+        } else if (mode == kModeInt) {
+            int32_t acc[kSrvVec];
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0;
+            for (int g = 0; g < ngroups; ++g) {
+                uint32_t wv[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int w = g * 8 + i;
+                    wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                }
+                uint32_t lo, hi;
+                gather_bytes(wv, bsel, lo, hi);
+                transpose8x8(lo, hi);
+                const int32_t* L = ilut + g * 256;
+#pragma unroll
+                for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
             }
-        }
-        float z[4];
-        uint32_t nib = 0u;
 #pragma unroll
-        for (int c = 0; c < kVec; ++c) {
-            const float y = __double2float_rn(__ddiv_rn(acc[c], dW));
-            const float e = __fsub_rn(zp[c], zp[c] >= 0.0f ? Sp : -Sp);
-            const float zv = c < nv ? __fadd_rn(y, e) : 0.0f;
+            for (int c = 0; c < kSrvVec; ++c)
+                y[c] = POW2 ? __int2float_rn(acc[c]) * ykscale
+                            : __double2float_rn(__ddiv_rn((double)acc[c] * unit, dW));
+        } else if (mode == kModeF64) {
+            double acc[kSrvVec];
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
+            for (int g = 0; g < ngroups; ++g) {
+                uint32_t wv[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int w = g * 8 + i;
+                    wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                }
+                uint32_t lo, hi;
+                gather_bytes(wv, bsel, lo, hi);
+                transpose8x8(lo, hi);
+                const double* L = lut + g * 256;
+#pragma unroll
+                for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], L[byte_of(lo, hi, c)]);
+            }
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
+        } else {
+            double acc[kSrvVec];
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
+            for (int w = 0; w < W; ++w) {
+                const uint32_t byte = nv > 0 ? (tw[w * kTileRow] >> (8 * bsel)) : 0u;
+                const double sv = sw[w];
+#pragma unroll
+                for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], ((byte >> c) & 1u) ? sv : -sv);
+            }
+#pragma unroll
+            for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
+        }
+        float z[kSrvVec];
+        uint32_t byte = 0u;
+#pragma unroll
+        for (int c = 0; c < kSrvVec; ++c) {
+            const float e = __fsub_rn(zp[it][c], zp[it][c] >= 0.0f ? Sp : -Sp);
+            const float zv = c < nv ? __fadd_rn(y[c], e) : 0.0f;
             z[c] = zv;
-            nib |= (c < nv && zv >= 0.0f) ? (1u << c) : 0u;
+            byte |= (c < nv && zv >= 0.0f) ? (1u << c) : 0u;
             nan_seen |= (zv != zv);
             ss = __fma_rn((double)zv, (double)zv, ss);
         }
-        if (nv > 0) st4(a.es + base + off, z);
-        const uint32_t word = gather_word(nib, lane);
-        if ((lane & 7) == 0 && nv > 0) a.bits_s[(base >> 5) + (q >> 3)] = word;
+        if (nv > 0) {
+            const float h0[4] = {z[0], z[1], z[2], z[3]}, h1[4] = {z[4], z[5], z[6], z[7]};
+            st4(a.es + base + off, h0);
+            st4(a.es + base + off + 4, h1);
+        }
+        uint32_t word = byte << (8 * (lane & 3));
+        word |= __shfl_xor_sync(kFull, word, 1);
+        word |= __shfl_xor_sync(kFull, word, 2);
+        if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
     }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
-    if (tid == 0) a.part_s[k * a.geo.nseg + j] = block_total(red);
+    if (tid == 0) a.part_s[k * a.geo.nseg_s + j] = block_total(red);
     if (__syncthreads_or(nan_seen) && tid == 0) atomicOr(a.status, kNanServer);
 }
 
@@ -342,7 +643,7 @@ struct ApplyArgs {
 
 __global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
     int64_t k, j, base, len;
-    if (!block_segment(a.geo, k, j, base, len)) return;
+    if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x, lane = tid & 31;
     const float S = a.S[k];
     const int sh = 4 * (lane & 7);
@@ -384,7 +685,7 @@ struct WarmupArgs {
 template <typename GT, bool VEC>
 __global__ void __launch_bounds__(kThreads) k_warmup(const WarmupArgs a) {
     int64_t k, j, base, len;
-    if (!block_segment(a.geo, k, j, base, len)) return;
+    if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
     const double dW = (double)a.geo.W;

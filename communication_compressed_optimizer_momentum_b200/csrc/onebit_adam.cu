@@ -100,7 +100,7 @@ Layout make_layout(const onebit_adam_s& h) {
     L.S_out = take(g.nch * f);
     L.S_lazy = take(g.nch * f);
     L.part_w = take((uint64_t)g.W * g.nch * g.nseg * sizeof(double));
-    L.part_s = take((uint64_t)g.nch * g.nseg * sizeof(double));
+    L.part_s = take((uint64_t)g.nch * g.nseg_s * sizeof(double));
     L.status = take(4 * sizeof(uint32_t));
     L.total = off;
     return L;
@@ -109,20 +109,22 @@ Layout make_layout(const onebit_adam_s& h) {
 bool valid_handle(onebit_adam_t h) { return h != nullptr; }
 
 int64_t step_blocks(const Geometry& g) { return g.nch * g.nseg; }
+int64_t server_blocks(const Geometry& g) { return g.nch * g.nseg_s; }
 
-// Launch the chunk-scale reduction with the thread count that fits the partial count.
-int launch_scales(const Geometry& g, const double* part, int64_t rows, float* out, float* lazy,
-                  cudaStream_t st) {
+// Launch the chunk-scale reduction (nseg partials of seg elements per row) with the thread
+// count that fits the partial count.
+int launch_scales(const Geometry& g, const double* part, int64_t rows, int64_t nseg, int seg,
+                  float* out, float* lazy, cudaStream_t st) {
     if (rows == 0) return ONEBIT_OK;
-    if (g.nseg <= 8) {
+    if (nseg <= 8) {
         k_scales<1><<<(unsigned)ceil_div(rows, kThreads), kThreads, 0, st>>>(
-            part, rows, g.nch, g.nseg, g.C, g.d, out, lazy);
-    } else if (g.nseg <= 1024) {
+            part, rows, g.nch, nseg, seg, g.C, g.d, out, lazy);
+    } else if (nseg <= 1024) {
         k_scales<32><<<(unsigned)ceil_div(rows, kWarps), kThreads, 0, st>>>(
-            part, rows, g.nch, g.nseg, g.C, g.d, out, lazy);
+            part, rows, g.nch, nseg, seg, g.C, g.d, out, lazy);
     } else {
-        k_scales<kThreads><<<(unsigned)rows, kThreads, 0, st>>>(part, rows, g.nch, g.nseg, g.C,
-                                                                g.d, out, lazy);
+        k_scales<kThreads><<<(unsigned)rows, kThreads, 0, st>>>(part, rows, g.nch, nseg, seg,
+                                                                g.C, g.d, out, lazy);
     }
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
@@ -220,6 +222,7 @@ int onebit_adam_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float 
     g.C = C;
     g.nch = ceil_div(d, C);
     g.nseg = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSeg);
+    g.nseg_s = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSegS);
     g.ld = round_up(d > 0 ? d : 1, 64);
     h->nw = ceil_div(d, 32);
     g.ldw = round_up(h->nw > 0 ? h->nw : 1, 4);
@@ -265,6 +268,9 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->part_s = reinterpret_cast<double*>(b + L.part_s);
     h->status = reinterpret_cast<uint32_t*>(b + L.status);
     h->gtype = grad_dtype;
+    const int ssm = (int)server_smem_bytes(h->geo.W);
+    ONEBIT_CUDA(cudaFuncSetAttribute(k_server<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
+    ONEBIT_CUDA(cudaFuncSetAttribute(k_server<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     cudaStream_t st = as_stream(stream);
     // m and v start at zero (Adam); the rest is cleared too so padding is deterministic.
     ONEBIT_CUDA(cudaMemsetAsync(b, 0, L.total, st));
@@ -317,14 +323,19 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
                                  : launch_worker<float>(h, grads, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 1, st);
-    rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, h->s_out, h->s_lazy, st);
+    rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out, h->s_lazy, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 2, st);
     ServerArgs sa{g, h->bits_w, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s, h->status};
-    k_server<<<blocks, kThreads, (size_t)(g.W + kWarps) * sizeof(double), st>>>(sa);
+    const size_t ssm = server_smem_bytes(g.W);
+    const unsigned sblocks = (unsigned)server_blocks(g);
+    if ((g.W & (g.W - 1)) == 0)
+        k_server<true><<<sblocks, kThreads, ssm, st>>>(sa);
+    else
+        k_server<false><<<sblocks, kThreads, ssm, st>>>(sa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 3, st);
-    rc = launch_scales(g, h->part_s, g.nch, h->S_out, h->S_lazy, st);
+    rc = launch_scales(g, h->part_s, g.nch, g.nseg_s, kSegS, h->S_out, h->S_lazy, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 4, st);
     ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, h->m, x};

@@ -43,6 +43,7 @@ class Workload:
     seed: int
     layer_sizes: Tuple[int, ...] = ()   # segment lengths whose sigma is drawn per segment
     lr: float = LR
+    last_worker_sigma: float = 1.0   # sigma multiplier of the last worker (scale-spread cases)
     beta1: float = BETA1
     beta2: float = BETA2
     eps: float = EPS
@@ -213,7 +214,8 @@ def np_grads(wl: Workload, phase: int, step: int) -> np.ndarray:
     rows = []
     for w in range(wl.W):
         rng = np.random.default_rng(step_seed(wl, phase, step, w))
-        rows.append(_np_worker_grad(wl, rng, sig))
+        mult = wl.last_worker_sigma if w == wl.W - 1 else 1.0
+        rows.append((_np_worker_grad(wl, rng, sig) * np.float32(mult)).astype(np.float32))
     g = np.stack(rows)
     return f32_to_bf16_bits(g) if wl.grad_dtype == "bf16" else g
 
@@ -272,6 +274,8 @@ def torch_fill_grads(wl: Workload, out, phase: int, step: int, piece: int = 1 <<
                     near = torch.rand(n, device=dev, generator=gen).mul_(2e-9).sub_(1e-9)
                     g = torch.where(u < 0.001, torch.zeros_like(g), g)
                     g = torch.where((u >= 0.001) & (u < 0.002), near, g)
+            if w == wl.W - 1 and wl.last_worker_sigma != 1.0:
+                g = g * wl.last_worker_sigma
             out[w, lo:hi].copy_(g)   # float32 -> bfloat16 rounds to nearest even
 
 
