@@ -192,6 +192,22 @@ def onebit_unpack(words, scales, n: int, C: int, out=None, stream=None):
     return out
 
 
+def onebit_compress_static(x, C: int, words=None, scales=None, stream=None):
+    """Sign words and per-chunk scales of a float32 CUDA tensor, computed without any device
+    allocation inside the library (its scratch is a fixed array in the library). For callers
+    that cannot allocate, pass preallocated ``words`` (int32, ceil(n/32)) and ``scales``
+    (float32, ceil(n/C)); the defaults here allocate them with torch for convenience."""
+    import torch
+    n = x.numel()
+    if words is None:
+        words = torch.empty((n + 31) // 32, dtype=torch.int32, device=x.device)
+    if scales is None:
+        scales = torch.empty((n + C - 1) // C, dtype=torch.float32, device=x.device)
+    _check(_abi.lib().onebit_compress_static(_ptr(x), n, C, _ptr(words), _ptr(scales),
+                                             _stream(stream)), "onebit_compress_static")
+    return words, scales
+
+
 # ----------------------------------------------------------------------------------------------
 # convenience owner of one handle + workspace
 

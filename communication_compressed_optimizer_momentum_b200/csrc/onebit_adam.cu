@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <string>
 #include <vector>
@@ -580,3 +581,113 @@ int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// One-vector compression whose scratch is a fixed array inside the library, so that neither the
+// caller nor the library allocates device memory for it.
+
+namespace {
+
+// fp64 norm partials of onebit_compress_static: one slot per kSeg-element segment, 512 KiB.
+// Every GPU that loads the library holds this array until the process exits.
+constexpr int64_t kStaticSegs = 1 << 16;
+static __device__ __align__(256) double g_static_partials[kStaticSegs];
+
+constexpr int kMaxDevices = 64;
+double* g_static_addr[kMaxDevices] = {};
+std::mutex g_static_mu;
+
+// Device address of g_static_partials on the current device, looked up once per device. In
+// host code the array's name is only a host-side stand-in, never a device address.
+int static_partials(double** out) {
+    int dev = 0;
+    ONEBIT_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return ONEBIT_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_addr[dev] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_static_partials);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_static_addr[dev] = static_cast<double*>(p);
+    }
+    *out = g_static_addr[dev];
+    return ONEBIT_OK;
+}
+
+// Sign words and per-segment fp64 sums of squares of x, one kSeg segment per block; the
+// per-thread, per-warp and per-block summation order is the worker kernel's, so the scales
+// equal the compressed step's worker scales for the same values.
+__global__ void __launch_bounds__(kThreads, 8) k_compress_partials(const float* x, int64_t n,
+                                                                   int64_t C, int64_t nseg,
+                                                                   uint32_t* words,
+                                                                   double* part) {
+    __shared__ double red[kWarps];
+    const int64_t k = (int64_t)blockIdx.x / nseg;
+    const int64_t j = (int64_t)blockIdx.x - k * nseg;
+    const int64_t c0 = k * C;
+    const int64_t clen = min(C, n - c0);
+    const int64_t s0 = j * kSeg;
+    if (s0 >= clen) return;
+    const int64_t base = c0 + s0;
+    const int64_t len = min((int64_t)kSeg, clen - s0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    double ss = 0.0;
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+        const int q = it * kThreads + tid;
+        const int64_t off = (int64_t)q * kVec;
+        const int nv = valid_of(len, off);
+        float xv[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if (nv > 0) ld4_caller(x + base + off, nv, xv);
+        uint32_t nib = 0u;
+#pragma unroll
+        for (int c = 0; c < kVec; ++c) {
+            const float v = c < nv ? xv[c] : 0.0f;
+            nib |= (c < nv && v >= 0.0f) ? (1u << c) : 0u;
+            ss = __fma_rn((double)v, (double)v, ss);
+        }
+        const uint32_t word = gather_word(nib, lane);
+        if ((lane & 7) == 0 && nv > 0) words[(base >> 5) + (q >> 3)] = word;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) part[k * nseg + j] = block_total(red);
+}
+
+}  // namespace
+
+extern "C" int onebit_compress_static(const float* x, int64_t n, int64_t C, uint32_t* words,
+                                      float* scales, void* stream) {
+    if (n < 0 || C <= 0) return ONEBIT_ERR_ARG;
+    if (C % 32 != 0) return ONEBIT_ERR_ALIGN;
+    if (n == 0) return ONEBIT_OK;
+    if (x == nullptr || words == nullptr || scales == nullptr) return ONEBIT_ERR_ARG;
+    if (!aligned16(x) || (reinterpret_cast<uintptr_t>(words) & 3u) ||
+        (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return ONEBIT_ERR_ALIGN;
+    if (n > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
+    const int64_t nch = ceil_div(n, C);
+    const int64_t nseg = ceil_div(std::min(C, n), kSeg);
+    if (nch * nseg > kStaticSegs) {
+        g_last_error = "onebit_compress_static: ceil(n/C) * ceil(min(C,n)/2048) = " +
+                       std::to_string(nch * nseg) + " segments exceeds the fixed scratch of " +
+                       std::to_string(kStaticSegs);
+        return ONEBIT_ERR_SPACE;
+    }
+    double* part = nullptr;
+    const int rc = static_partials(&part);
+    if (rc != ONEBIT_OK) return rc;
+    cudaStream_t st = as_stream(stream);
+    k_compress_partials<<<(unsigned)(nch * nseg), kThreads, 0, st>>>(x, n, C, nseg, words, part);
+    ONEBIT_CUDA(cudaGetLastError());
+    Geometry g{};
+    g.d = n;
+    g.C = C;
+    g.nch = nch;
+    g.nseg = nseg;
+    g.W = 1;
+    // every slot read by the reduction was written by k_compress_partials in this same call,
+    // so nothing in the shared array has to be cleared first
+    return launch_scales(g, part, nch, nseg, kSeg, scales, scales, st);
+}

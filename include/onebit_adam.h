@@ -201,6 +201,30 @@ int onebit_pack(const float* x, int64_t n, uint32_t* words, void* stream);
 int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t C, float* out,
                   void* stream);
 
+/*
+ * Compress one fp32 vector x[n] (device) into its 1-bit message: LSB-first sign words
+ * words[ceil(n/32)] (bit = x >= 0) and one scale per chunk of C elements,
+ * scales[ceil(n/C)] = sqrt(sum of squares / chunk length) -- the worker compression of the
+ * compressed step applied to x itself. The paper has no counterpart of this entry point: it is
+ * the library's variant of that kernel for callers that must not allocate device memory, for
+ * example code running inside a host application or plugin that hands it only its input and
+ * output buffers and owns the whole device memory pool, or latency-critical paths where the
+ * implicit synchronisation of cudaMalloc/cudaFree is not acceptable. It allocates nothing: its
+ * scratch (the fp64 norm partials) is a fixed 512 KiB array inside the library, which every GPU
+ * that loads the library keeps until the process exits.
+ *   Limit: ceil(n/C) * ceil(min(C, n)/2048) <= 65536 (for example n <= 134,217,728 when C is a
+ *   multiple of 2048); larger inputs return ONEBIT_ERR_SPACE with the reason in
+ *   onebit_last_error(), before any device work.
+ *   C >= 32, C % 32 == 0 (ONEBIT_ERR_ALIGN otherwise); x 16-byte aligned; n = 0 is a no-op.
+ *   The first call on each device looks up the array's device address (with that device
+ *   current) and caches it; make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents; each call writes every
+ *   slot it reads before reading it. Calls whose work overlaps on the GPU (for example on two
+ *   streams at once) race on the array and must be ordered by the caller.
+ */
+int onebit_compress_static(const float* x, int64_t n, int64_t C, uint32_t* words, float* scales,
+                           void* stream);
+
 /* Static description of a status code. */
 const char* onebit_strerror(int32_t code);
 
