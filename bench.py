@@ -167,6 +167,22 @@ class ClockSampler:
                 "in_timed_region": bool(inside)}
 
 
+def max_over_ranks(value, device):
+    """The max of a per-rank number over all ranks of the default process group (the number
+    itself with one rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms_max):
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def _to_np(t):
     import numpy as np
     import torch
@@ -249,14 +265,10 @@ def run_ours(args):
     opt.timing(0)
     time.sleep(0.3)
     clocks = sampler.stop()
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dev)
     status = opt.status()
 
-    units = wl.d * wl.W * args.steps * world
-    value = units / (ms_max / 1e3)
+    value = whole_job_rate(wl.d * wl.W * args.steps, world, ms_max)
     step_bytes = wl.algorithmic_bytes_per_param() * wl.d
     achieved_step_gbs = step_bytes * args.steps / (ms_max / 1e3) / 1e9
     peak, peak_src = measured_hbm_peak()
@@ -282,10 +294,8 @@ def run_ours(args):
             opt.step_host(x, g, g_host, x_host, wl.lr)
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e2e = {"value": wl.d * wl.W * args.e2e_steps * world / (float(e_ms.item()) / 1e3),
+        e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": whole_job_rate(wl.d * wl.W * args.e2e_steps, world, e_ms),
                "unit": UNIT, "steps": args.e2e_steps,
                "h2d_bytes_per_step": wl.W * wl.d * wl.grad_bytes,
                "d2h_bytes_per_step": wl.d * 4}
