@@ -158,7 +158,9 @@ __device__ __forceinline__ double block_total(const double* red) {
 struct WorkerArgs {
     Geometry geo;
     float beta1, omb1;
-    const float* m;       // [ld] library-owned
+    const float* m;       // [ld] explicit momentum (first step after freeze or set_state)
+    const uint32_t* bits_s;  // [ldw] previous step's server plane: m = +-S (later steps)
+    const float* S;          // [nch] previous step's server scales
     const void* g;        // [W][d] caller-owned, GT
     float* ew;            // [W][ld] lazy residual: holds last step's x_w
     const float* s_lazy;  // [W][nch] scale that rebuilds the residual
@@ -169,7 +171,10 @@ struct WorkerArgs {
 
 // 8 resident blocks per SM (at most 32 registers a thread): the kernel is latency-bound on HBM
 // and more warps in flight beat deeper per-thread prefetch (measured on B200).
-template <typename GT, bool VEC>
+// LAZY_M: the shared momentum is the decompressed server message of the previous step, m =
+// (bit ? S_k : -S_k), rebuilt here from the server plane instead of read as fp32 (4 bytes per
+// parameter fewer to read, and k_apply need not write it).
+template <typename GT, bool VEC, bool LAZY_M>
 __global__ void __launch_bounds__(kThreads, 8) k_worker(const WorkerArgs a) {
     extern __shared__ double red_w[];  // [W][kWarps]
     int64_t k, j, base, len;
@@ -183,8 +188,18 @@ __global__ void __launch_bounds__(kThreads, 8) k_worker(const WorkerArgs a) {
     for (int it = 0; it < kItems; ++it) {
         const int64_t off = (int64_t)(it * kThreads + tid) * kVec;
         nv[it] = valid_of(len, off);
-        if (nv[it] > 0) ld4(a.m + base + off, mr[it]);
-        else { mr[it][0] = mr[it][1] = mr[it][2] = mr[it][3] = 0.0f; }
+        if (nv[it] > 0) {
+            if (LAZY_M) {
+                const float S = a.S[k];
+                const uint32_t nib = a.bits_s[(base >> 5) + ((it * kThreads + tid) >> 3)] >> (4 * (lane & 7));
+#pragma unroll
+                for (int c = 0; c < kVec; ++c) mr[it][c] = ((nib >> c) & 1u) ? S : -S;
+            } else {
+                ld4(a.m + base + off, mr[it]);
+            }
+        } else {
+            mr[it][0] = mr[it][1] = mr[it][2] = mr[it][3] = 0.0f;
+        }
     }
     const float b1 = a.beta1, omb1 = a.omb1;
     bool nan_seen = false;
@@ -312,14 +327,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 }
 
 // ------------------------------------------------------------------------------------------
-// K2: the server side of the compressed allreduce for one kSegS segment of chunk k.
+// K2: the server side of the compressed allreduce. Per element of chunk k:
 //   y = fl32(fp64 sum_w (+-s_w,k) / W);  z = y + e_s;  bit = z >= 0;
 //   store z (lazy server residual);  fp64 partial of sum z^2.
 // LIT-278 note, Key takeaways and "What the evidence does not cover" (the compressed allreduce).
 //
-// Staging. Thread 0 starts one TMA bulk copy per worker (that worker's sign words of the
-// segment, at most 512 bytes) into shared memory; while they land, the block loads the scales,
-// checks exactness and builds its lookup tables, and every thread fetches its residuals.
+// Work split. A block owns up to kSrvSegsPerBlock consecutive kSegS-element segments of one
+// chunk: it reads the chunk's W scales, picks the decode mode and builds its lookup tables once,
+// then streams its segments. Each segment's W plane rows (at most 528 bytes each) arrive in
+// shared memory by TMA bulk copies counted on a per-stage mbarrier; with two stages the copies
+// of segment t + 2 are in flight while segment t is decoded. Residuals are read and z written
+// with plain 16-byte accesses.
 //
 // Decoding. Thread t owns 8 consecutive elements: byte (t % 4) of one 32-element word of every
 // worker's plane. For each group of 8 workers it gathers their 8 bytes (__byte_perm), transposes
@@ -336,6 +354,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
 
 enum ServerMode : int { kModeY = 0, kModeInt = 1, kModeF64 = 2, kModeSeq = 3 };
 
+constexpr int kSrvSegsPerBlock = 8;        // server segments per block
 constexpr int kSegWords = kSegS / 32;      // sign words per worker per server segment
 constexpr int kTileRow = kSegWords + 4;    // staged row: the segment's words plus up to 3 words
                                            // before them (copies start 16-byte aligned)
@@ -351,11 +370,17 @@ struct ServerArgs {
     uint32_t* status;
 };
 
-// Dynamic shared memory of k_server for W workers (bytes).
-__host__ __device__ inline size_t server_smem_bytes(int W) {
+// Pipeline depth of k_server: two stages while they fit next to the tables and a block has
+// more than one segment to stream.
+__host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
+    return (W <= 128 && nseg_s > 1) ? 2 : 1;
+}
+
+// Dynamic shared memory of k_server for W workers and `nst` stages (bytes).
+__host__ __device__ inline size_t server_smem_bytes(int W, int nst) {
     const int wpad = (W + 7) & ~7;
-    return 32                                                   // mbarrier, mode, unit
-         + (size_t)W * kTileRow * sizeof(uint32_t)              // staged sign words
+    return 64                                                   // mbarriers, mode, unit
+         + (size_t)nst * W * kTileRow * sizeof(uint32_t)        // staged sign words
          + (size_t)wpad * sizeof(double)                        // scales
          + (size_t)(wpad / 8) * 256 * sizeof(double)            // per-group tables
          + 256 * sizeof(float)                                  // y table (W <= 8)
@@ -392,59 +417,58 @@ __device__ __forceinline__ float server_average(double acc, double dW, double in
     return __double2float_rn(POW2 ? acc * invW : __ddiv_rn(acc, dW));
 }
 
+// Start the bulk copies of segment j's W plane rows into one stage (thread 0 only).
+__device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stage,
+                                             uint64_t* bar, int64_t c0, int64_t clen,
+                                             int64_t j) {
+    const int64_t base = c0 + j * kSegS;
+    const int64_t len = min((int64_t)kSegS, clen - j * kSegS);
+    const int64_t wbase = base >> 5;
+    // words [wbase & ~3, round_up(wbase + ceil(len / 32), 4)) of each row: both ends 16-byte
+    // aligned and inside the row (plane rows are padded to a multiple of 4 words)
+    const int lead = (int)(wbase & 3);
+    const uint32_t row_bytes = (uint32_t)(((lead + (len + 31) / 32 + 3) / 4) * 16);
+    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)a.geo.W);
+    for (int w = 0; w < a.geo.W; ++w)
+        bulk_load(stage + (size_t)w * kTileRow,
+                  a.bits_w + (int64_t)w * a.geo.ldw + (wbase - lead), row_bytes, bar);
+}
+
 template <bool POW2>
 __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     extern __shared__ __align__(16) unsigned char smem_srv[];
-    int64_t k, j, base, len;
-    if (!block_segment<kSegS>(a.geo, a.geo.nseg_s, k, j, base, len)) return;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = a.geo.W;
+    const int64_t nsb = (a.geo.nseg_s + kSrvSegsPerBlock - 1) / kSrvSegsPerBlock;
+    const int64_t k = (int64_t)blockIdx.x / nsb;
+    const int64_t b = (int64_t)blockIdx.x - k * nsb;
+    const int64_t c0 = k * a.geo.C;
+    const int64_t clen = min(a.geo.C, a.geo.d - c0);
+    const int64_t nseg_k = (clen + kSegS - 1) / kSegS;
+    const int64_t j0 = b * kSrvSegsPerBlock;
+    if (j0 >= nseg_k) return;
+    const int nseg_blk = (int)min((int64_t)kSrvSegsPerBlock, nseg_k - j0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wpad = (W + 7) & ~7, ngroups = wpad / 8;
-    uint64_t* bar = reinterpret_cast<uint64_t*>(smem_srv);
-    int* mode_p = reinterpret_cast<int*>(smem_srv + 8);
-    int* emin_p = reinterpret_cast<int*>(smem_srv + 12);    // smallest effective exponent
-    double* unit_p = reinterpret_cast<double*>(smem_srv + 16);
-    uint32_t* tile = reinterpret_cast<uint32_t*>(smem_srv + 32);         // [W][kTileRow]
-    double* sw = reinterpret_cast<double*>(tile + (size_t)W * kTileRow);
+    const int nst = server_stages(W, a.geo.nseg_s);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_srv);             // [nst] (<= 2)
+    int* mode_p = reinterpret_cast<int*>(smem_srv + 16);
+    int* emin_p = reinterpret_cast<int*>(smem_srv + 20);     // smallest effective exponent
+    double* unit_p = reinterpret_cast<double*>(smem_srv + 24);
+    uint32_t* stages = reinterpret_cast<uint32_t*>(smem_srv + 64);      // [nst][W][kTileRow]
+    double* sw = reinterpret_cast<double*>(stages + (size_t)nst * W * kTileRow);
     double* lut = sw + wpad;                                  // fp64 tables [ngroups][256]
     int32_t* ilut = reinterpret_cast<int32_t*>(lut);          // or int32 tables, same place
     float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
     double* red = reinterpret_cast<double*>(ylut + 256);
     const double dW = (double)W, invW = 1.0 / (double)W;
-    const int64_t wbase = base >> 5;
-    // Copy words [wbase & ~3, round_up(wbase + ceil(len / 32), 4)) of every plane row: both ends
-    // 16-byte aligned and inside the row (rows are padded to a multiple of 4 words).
-    const int lead = (int)(wbase & 3);
-    const uint32_t row_bytes = (uint32_t)(((lead + (len + 31) / 32 + 3) / 4) * 16);
 
     if (tid == 0) {
-        mbar_init(bar, 1);
-        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)W);
-        for (int w = 0; w < W; ++w)
-            bulk_load(tile + (size_t)w * kTileRow,
-                      a.bits_w + (int64_t)w * a.geo.ldw + (wbase - lead), row_bytes, bar);
+        for (int st = 0; st < nst; ++st) mbar_init(&bars[st], 1);
+        for (int t = 0; t < nst && t < nseg_blk; ++t)
+            server_issue(a, stages + (size_t)t * W * kTileRow, &bars[t], c0, clen, j0 + t);
     }
     for (int w = tid; w < wpad; w += kThreads)
         sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
-    // residuals of this thread's elements, fetched while the copies are in flight
-    float zp[kSrvItems][kSrvVec];
-    int nvs[kSrvItems];
-#pragma unroll
-    for (int it = 0; it < kSrvItems; ++it) {
-        const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
-        const int64_t rem = len - off;
-        nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
-        if (nvs[it] > 0) {
-            float h0[4], h1[4];
-            ld4(a.es + base + off, h0);
-            ld4(a.es + base + off + 4, h1);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
-        } else {
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) zp[it][c] = 0.0f;
-        }
-    }
     __syncthreads();
     if (warp == 0) {
         // exactness bound over the W scales (warp-parallel, fixed reduction order)
@@ -514,120 +538,159 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
         }
     }
     __syncthreads();
-    if (!mbar_wait_bounded(bar, 0)) {
-        // the copies did not land in time: record it, give them one more bounded wait, leave
-        if (tid == 0) atomicOr(a.status, kWaitTimeout);
-        mbar_wait_bounded(bar, 0);
-        return;
-    }
     const float ykscale = __int_as_float((min(max(*emin_p - 150 - (__ffs(W) - 1), -126), 127) + 127) << 23);
     const double unit = *unit_p;
     const float Sp = a.S_lazy[k];
     double ss = 0.0;
     bool nan_seen = false;
+
+    for (int t = 0; t < nseg_blk; ++t) {
+        const int st = t % nst;
+        const uint32_t parity = (uint32_t)((t / nst) & 1);
+        const int64_t base = c0 + (j0 + t) * kSegS;
+        const int64_t len = min((int64_t)kSegS, clen - (j0 + t) * kSegS);
+        const int64_t wbase = base >> 5;
+        const int lead = (int)(wbase & 3);
+        // residuals first, so their latency overlaps the wait for the planes
+        float zp[kSrvItems][kSrvVec];
+        int nvs[kSrvItems];
 #pragma unroll
-    for (int it = 0; it < kSrvItems; ++it) {
-        const int q = it * kThreads + tid;            // 8-element group index in the segment
-        const int64_t off = (int64_t)q * kSrvVec;
-        const int nv = nvs[it];
-        const int wd = q >> 2, bsel = q & 3;           // word within the segment, byte within it
-        const uint32_t* tw = tile + lead + wd;
-        float y[kSrvVec];
-        if (mode == kModeY) {
-            uint32_t wv[8];
+        for (int it = 0; it < kSrvItems; ++it) {
+            const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
+            const int64_t rem = len - off;
+            nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
+            if (nvs[it] > 0) {
+                float h0[4], h1[4];
+                ld4(a.es + base + off, h0);
+                ld4(a.es + base + off + 4, h1);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) wv[i] = (i < W && nv > 0) ? tw[i * kTileRow] : 0u;
-            uint32_t lo, hi;
-            gather_bytes(wv, bsel, lo, hi);
-            transpose8x8(lo, hi);
+                for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
+            } else {
 #pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) y[c] = ylut[byte_of(lo, hi, c)];
-        } else if (mode == kModeInt) {
-            int32_t acc[kSrvVec];
+                for (int c = 0; c < kSrvVec; ++c) zp[it][c] = 0.0f;
+            }
+        }
+        const bool landed = mbar_wait_bounded(&bars[st], parity);
+        if (landed) {
+            const uint32_t* tile = stages + (size_t)st * W * kTileRow;
 #pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0;
-            for (int g = 0; g < ngroups; ++g) {
-                uint32_t wv[8];
+            for (int it = 0; it < kSrvItems; ++it) {
+                const int q = it * kThreads + tid;        // 8-element group index in the segment
+                const int64_t off = (int64_t)q * kSrvVec;
+                const int nv = nvs[it];
+                const int wd = q >> 2, bsel = q & 3;       // word within the segment, byte in it
+                const uint32_t* tw = tile + lead + wd;
+                float y[kSrvVec];
+                if (mode == kModeY) {
+                    uint32_t wv[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int w = g * 8 + i;
-                    wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                    for (int i = 0; i < 8; ++i) wv[i] = (i < W && nv > 0) ? tw[i * kTileRow] : 0u;
+                    uint32_t lo, hi;
+                    gather_bytes(wv, bsel, lo, hi);
+                    transpose8x8(lo, hi);
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) y[c] = ylut[byte_of(lo, hi, c)];
+                } else if (mode == kModeInt) {
+                    int32_t acc[kSrvVec];
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) acc[c] = 0;
+                    for (int g = 0; g < ngroups; ++g) {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int w = g * 8 + i;
+                            wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                        }
+                        uint32_t lo, hi;
+                        gather_bytes(wv, bsel, lo, hi);
+                        transpose8x8(lo, hi);
+                        const int32_t* L = ilut + g * 256;
+#pragma unroll
+                        for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
+                    }
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c)
+                        y[c] = POW2 ? __int2float_rn(acc[c]) * ykscale
+                                    : __double2float_rn(__ddiv_rn((double)acc[c] * unit, dW));
+                } else if (mode == kModeF64) {
+                    double acc[kSrvVec];
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
+                    for (int g = 0; g < ngroups; ++g) {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int w = g * 8 + i;
+                            wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                        }
+                        uint32_t lo, hi;
+                        gather_bytes(wv, bsel, lo, hi);
+                        transpose8x8(lo, hi);
+                        const double* L = lut + g * 256;
+#pragma unroll
+                        for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], L[byte_of(lo, hi, c)]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
+                } else {
+                    double acc[kSrvVec];
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
+                    for (int w = 0; w < W; ++w) {
+                        const uint32_t byte = nv > 0 ? (tw[w * kTileRow] >> (8 * bsel)) : 0u;
+                        const double sv = sw[w];
+#pragma unroll
+                        for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], ((byte >> c) & 1u) ? sv : -sv);
+                    }
+#pragma unroll
+                    for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
                 }
-                uint32_t lo, hi;
-                gather_bytes(wv, bsel, lo, hi);
-                transpose8x8(lo, hi);
-                const int32_t* L = ilut + g * 256;
+                float z[kSrvVec];
+                uint32_t byte = 0u;
 #pragma unroll
-                for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
-            }
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c)
-                y[c] = POW2 ? __int2float_rn(acc[c]) * ykscale
-                            : __double2float_rn(__ddiv_rn((double)acc[c] * unit, dW));
-        } else if (mode == kModeF64) {
-            double acc[kSrvVec];
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
-            for (int g = 0; g < ngroups; ++g) {
-                uint32_t wv[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int w = g * 8 + i;
-                    wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
+                for (int c = 0; c < kSrvVec; ++c) {
+                    const float e = __fsub_rn(zp[it][c], zp[it][c] >= 0.0f ? Sp : -Sp);
+                    const float zv = c < nv ? __fadd_rn(y[c], e) : 0.0f;
+                    z[c] = zv;
+                    byte |= (c < nv && zv >= 0.0f) ? (1u << c) : 0u;
+                    nan_seen |= (zv != zv);
+                    ss = __fma_rn((double)zv, (double)zv, ss);
                 }
-                uint32_t lo, hi;
-                gather_bytes(wv, bsel, lo, hi);
-                transpose8x8(lo, hi);
-                const double* L = lut + g * 256;
-#pragma unroll
-                for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], L[byte_of(lo, hi, c)]);
+                if (nv > 0) {
+                    const float h0[4] = {z[0], z[1], z[2], z[3]}, h1[4] = {z[4], z[5], z[6], z[7]};
+                    st4(a.es + base + off, h0);
+                    st4(a.es + base + off + 4, h1);
+                }
+                uint32_t word = byte << (8 * (lane & 3));
+                word |= __shfl_xor_sync(kFull, word, 1);
+                word |= __shfl_xor_sync(kFull, word, 2);
+                if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
             }
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
-        } else {
-            double acc[kSrvVec];
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
-            for (int w = 0; w < W; ++w) {
-                const uint32_t byte = nv > 0 ? (tw[w * kTileRow] >> (8 * bsel)) : 0u;
-                const double sv = sw[w];
-#pragma unroll
-                for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], ((byte >> c) & 1u) ? sv : -sv);
+        }
+        // everyone is done with this stage (or some thread's wait expired: then all leave,
+        // after one more bounded wait for the copies still in flight)
+        if (__syncthreads_or(!landed)) {
+            if (tid == 0) {
+                atomicOr(a.status, kWaitTimeout);
+                for (int u = t; u < nseg_blk && u < t + nst; ++u)
+                    mbar_wait_bounded(&bars[u % nst], (uint32_t)((u / nst) & 1));
             }
-#pragma unroll
-            for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
+            return;
         }
-        float z[kSrvVec];
-        uint32_t byte = 0u;
-#pragma unroll
-        for (int c = 0; c < kSrvVec; ++c) {
-            const float e = __fsub_rn(zp[it][c], zp[it][c] >= 0.0f ? Sp : -Sp);
-            const float zv = c < nv ? __fadd_rn(y[c], e) : 0.0f;
-            z[c] = zv;
-            byte |= (c < nv && zv >= 0.0f) ? (1u << c) : 0u;
-            nan_seen |= (zv != zv);
-            ss = __fma_rn((double)zv, (double)zv, ss);
-        }
-        if (nv > 0) {
-            const float h0[4] = {z[0], z[1], z[2], z[3]}, h1[4] = {z[4], z[5], z[6], z[7]};
-            st4(a.es + base + off, h0);
-            st4(a.es + base + off + 4, h1);
-        }
-        uint32_t word = byte << (8 * (lane & 3));
-        word |= __shfl_xor_sync(kFull, word, 1);
-        word |= __shfl_xor_sync(kFull, word, 2);
-        if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
+        if (tid == 0 && t + nst < nseg_blk)
+            server_issue(a, stages + (size_t)st * W * kTileRow, &bars[st], c0, clen, j0 + t + nst);
     }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
-    if (tid == 0) a.part_s[k * a.geo.nseg_s + j] = block_total(red);
+    if (tid == 0) a.part_s[k * nsb + b] = block_total(red);
     if (__syncthreads_or(nan_seen) && tid == 0) atomicOr(a.status, kNanServer);
 }
 
 // ------------------------------------------------------------------------------------------
 // K3: every worker decompresses the server message into the shared momentum and steps with
-// the frozen variance: m = (bit ? S_k : -S_k);  x -= lr * (m / (sqrt(v) + eps)).
+// the frozen variance: m = (bit ? S_k : -S_k);  x -= lr * (m / (sqrt(v) + eps)). The momentum
+// is kept in its compressed form (the server plane and S), which is exactly m.
 // "1-bit Adam" index page, Abstract (variance as a fixed preconditioner); LIT-278 note, Key
 // takeaways.
 
@@ -637,7 +700,6 @@ struct ApplyArgs {
     const uint32_t* bits_s;  // [ldw]
     const float* S;          // [nch]
     const float* v;          // [ld]
-    float* m;                // [ld]
     float* x;                // [d] caller-owned
 };
 
@@ -654,7 +716,7 @@ __global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
         const int nv = valid_of(len, off);
         if (nv == 0) continue;
         const uint32_t nib = a.bits_s[(base >> 5) + (q >> 3)] >> sh;
-        float v[4], x[4], m[4];
+        float v[4], x[4], m[4];  // m stays in registers: the next step rebuilds it from the plane
         ld4(a.v + base + off, v);
         ld4_caller(a.x + base + off, nv, x);
 #pragma unroll
@@ -664,7 +726,6 @@ __global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
             const float upd = __fmul_rn(a.lr, __fdiv_rn(m[c], den));
             x[c] = __fsub_rn(x[c], upd);
         }
-        st4(a.m + base + off, m);
         st4_caller(a.x + base + off, nv, x);
     }
 }

@@ -65,6 +65,7 @@ struct onebit_adam_s {
     float beta1, beta2, eps;
     int phase = kUnbound;
     int64_t steps = 0;
+    bool m_explicit = true;  // m in the fp32 buffer; else m = +-S_out by the server plane
     int32_t gtype = -1;
     char* ws = nullptr;
     Layout lay{};
@@ -110,7 +111,10 @@ Layout make_layout(const onebit_adam_s& h) {
 bool valid_handle(onebit_adam_t h) { return h != nullptr; }
 
 int64_t step_blocks(const Geometry& g) { return g.nch * g.nseg; }
-int64_t server_blocks(const Geometry& g) { return g.nch * g.nseg_s; }
+int64_t server_blocks_per_chunk(const Geometry& g) {
+    return ceil_div(g.nseg_s, kSrvSegsPerBlock);
+}
+int64_t server_blocks(const Geometry& g) { return g.nch * server_blocks_per_chunk(g); }
 
 // Launch the chunk-scale reduction (nseg partials of seg elements per row) with the thread
 // count that fits the partial count.
@@ -131,16 +135,35 @@ int launch_scales(const Geometry& g, const double* part, int64_t rows, int64_t n
     return ONEBIT_OK;
 }
 
+template <typename GT, bool LAZY_M>
+void launch_worker_t(onebit_adam_s* h, const WorkerArgs& a, unsigned blocks, size_t smem,
+                     cudaStream_t st) {
+    if (h->geo.d % kVec == 0)
+        k_worker<GT, true, LAZY_M><<<blocks, kThreads, smem, st>>>(a);
+    else
+        k_worker<GT, false, LAZY_M><<<blocks, kThreads, smem, st>>>(a);
+}
+
 template <typename GT>
 int launch_worker(onebit_adam_s* h, const void* grads, cudaStream_t st) {
-    WorkerArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->m, grads, h->ew, h->s_lazy, h->bits_w,
-                 h->part_w, h->status};
+    WorkerArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->m, h->bits_s, h->S_out, grads, h->ew,
+                 h->s_lazy, h->bits_w, h->part_w, h->status};
     const size_t smem = (size_t)h->geo.W * kWarps * sizeof(double);
     const unsigned blocks = (unsigned)step_blocks(h->geo);
-    if (h->geo.d % kVec == 0)
-        k_worker<GT, true><<<blocks, kThreads, smem, st>>>(a);
+    if (h->m_explicit)
+        launch_worker_t<GT, false>(h, a, blocks, smem, st);
     else
-        k_worker<GT, false><<<blocks, kThreads, smem, st>>>(a);
+        launch_worker_t<GT, true>(h, a, blocks, smem, st);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+// m = +-S_out by the server plane, for elements [i0, i0 + n) (chunk-aligned i0), into dst.
+int launch_materialize_m(onebit_adam_s* h, int64_t i0, int64_t n, float* dst, cudaStream_t st) {
+    if (n == 0) return ONEBIT_OK;
+    const Geometry& g = h->geo;
+    k_unpack<<<(unsigned)ceil_div(n, kSeg), kThreads, 0, st>>>(h->bits_s + i0 / 32,
+                                                               h->S_out + i0 / g.C, n, g.C, dst);
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }
@@ -269,7 +292,7 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->part_s = reinterpret_cast<double*>(b + L.part_s);
     h->status = reinterpret_cast<uint32_t*>(b + L.status);
     h->gtype = grad_dtype;
-    const int ssm = (int)server_smem_bytes(h->geo.W);
+    const int ssm = (int)server_smem_bytes(h->geo.W, server_stages(h->geo.W, h->geo.nseg_s));
     ONEBIT_CUDA(cudaFuncSetAttribute(k_server<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     ONEBIT_CUDA(cudaFuncSetAttribute(k_server<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     cudaStream_t st = as_stream(stream);
@@ -277,6 +300,7 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     ONEBIT_CUDA(cudaMemsetAsync(b, 0, L.total, st));
     h->phase = kWarmup;
     h->steps = 0;
+    h->m_explicit = true;
     return ONEBIT_OK;
 }
 
@@ -328,7 +352,7 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
     if (rc != ONEBIT_OK) return rc;
     record(h, 2, st);
     ServerArgs sa{g, h->bits_w, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s, h->status};
-    const size_t ssm = server_smem_bytes(g.W);
+    const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
     const unsigned sblocks = (unsigned)server_blocks(g);
     if ((g.W & (g.W - 1)) == 0)
         k_server<true><<<sblocks, kThreads, ssm, st>>>(sa);
@@ -336,15 +360,17 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
         k_server<false><<<sblocks, kThreads, ssm, st>>>(sa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 3, st);
-    rc = launch_scales(g, h->part_s, g.nch, g.nseg_s, kSegS, h->S_out, h->S_lazy, st);
+    rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
+                       kSegS * kSrvSegsPerBlock, h->S_out, h->S_lazy, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 4, st);
-    ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, h->m, x};
+    ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, x};
     k_apply<<<blocks, kThreads, 0, st>>>(pa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 5, st);
     if (h->tcount < h->tmax) ++h->tcount;
     ++h->steps;
+    h->m_explicit = false;  // m is now the server message of this step
     return ONEBIT_OK;
 }
 
@@ -395,7 +421,10 @@ int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* strea
     const Geometry& g = h->geo;
     const auto D2D = cudaMemcpyDeviceToDevice;
     switch (which) {
-        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m, bytes, D2D, st)); break;
+        case ONEBIT_STATE_M:
+            if (!h->m_explicit) return launch_materialize_m(h, 0, g.d, static_cast<float*>(dst), st);
+            ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m, bytes, D2D, st));
+            break;
         case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->v, bytes, D2D, st)); break;
         case ONEBIT_STATE_SW: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->s_out, bytes, D2D, st)); break;
         case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out, bytes, D2D, st)); break;
@@ -429,7 +458,10 @@ int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void*
     const uint64_t f = sizeof(float), u = sizeof(uint32_t);
     const auto D2D = cudaMemcpyDeviceToDevice;
     switch (which) {
-        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m + i0, n * f, D2D, st)); break;
+        case ONEBIT_STATE_M:
+            if (!h->m_explicit) return launch_materialize_m(h, i0, n, static_cast<float*>(dst), st);
+            ONEBIT_CUDA(cudaMemcpyAsync(dst, h->m + i0, n * f, D2D, st));
+            break;
         case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->v + i0, n * f, D2D, st)); break;
         case ONEBIT_STATE_EW:
         case ONEBIT_STATE_ES:
@@ -466,7 +498,10 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
     const auto D2D = cudaMemcpyDeviceToDevice;
     const uint64_t f = sizeof(float);
     switch (which) {
-        case ONEBIT_STATE_M: ONEBIT_CUDA(cudaMemcpyAsync(h->m, src, bytes, D2D, st)); break;
+        case ONEBIT_STATE_M:
+            ONEBIT_CUDA(cudaMemcpyAsync(h->m, src, bytes, D2D, st));
+            h->m_explicit = true;
+            break;
         case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(h->v, src, bytes, D2D, st)); break;
         case ONEBIT_STATE_EW:
             // explicit residual with a zero rebuild scale: e = stored - (+-0) = stored exactly
@@ -475,6 +510,12 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
             ONEBIT_CUDA(cudaMemsetAsync(h->s_out, 0, (uint64_t)g.W * g.nch * f, st));
             break;
         case ONEBIT_STATE_ES:
+            if (!h->m_explicit) {
+                // m lives in S_out, which is about to be cleared: make it explicit first
+                const int rc2 = launch_materialize_m(h, 0, g.d, h->m, st);
+                if (rc2 != ONEBIT_OK) return rc2;
+                h->m_explicit = true;
+            }
             ONEBIT_CUDA(cudaMemcpyAsync(h->es, src, bytes, D2D, st));
             ONEBIT_CUDA(cudaMemsetAsync(h->S_lazy, 0, g.nch * f, st));
             ONEBIT_CUDA(cudaMemsetAsync(h->S_out, 0, g.nch * f, st));

@@ -58,16 +58,19 @@ class Workload:
         return 4 if self.grad_dtype == "f32" else 2
 
     def algorithmic_bytes_per_param(self) -> float:
-        """Minimum HBM bytes per parameter for one compressed step when every state element is
-        read and written once and each message is written and read once:
-        W*(G + 4 + 4 + 1/8 + 1/8) + 8 (m) + 4 (v) + 8 (x) + 8 (server residual) + 1/4 (server
-        bits); the per-chunk scales are negligible and left out."""
-        return self.W * (self.grad_bytes + 8.25) + 28.25
+        """Minimum HBM bytes per parameter of one compressed step when every state element is
+        read and written once and each message is written and read once. Per worker: the
+        gradient (G), the residual read and written (4 + 4), its sign plane written and read
+        (1/8 + 1/8). Shared: the server residual read and written (8), the server plane written,
+        read by the apply and read again by the next step's worker pass, which rebuilds the
+        momentum m = +-S from it (3/8), v read (4), x read and written (8). Per-chunk scales
+        are negligible and left out: W*(G + 8.25) + 20.375."""
+        return self.W * (self.grad_bytes + 8.25) + 20.375
 
     def kernel_bytes_per_param(self) -> dict:
         """The same minimum, split by the three streaming kernels of the step."""
         G, W = self.grad_bytes, self.W
-        return {"worker": W * (G + 8.125) + 4.0, "server": W / 8.0 + 8.125, "apply": 16.125}
+        return {"worker": W * (G + 8.125) + 0.125, "server": W / 8.0 + 8.125, "apply": 12.125}
 
 
 def _ceil_to(x: int, a: int) -> int:

@@ -54,6 +54,8 @@ def padding_is_zero(words: np.ndarray, n: int) -> bool:
 
 
 def expand(scales: np.ndarray, C: int, n: int) -> np.ndarray:
+    if scales.shape[-1] == 1:          # one chunk: broadcast instead of materialising W x n
+        return np.broadcast_to(scales, scales.shape[:-1] + (n,))
     return np.repeat(scales, C, axis=-1)[..., :n]
 
 
@@ -152,7 +154,7 @@ POST = ("x", "m", "e_w", "e_s", "s", "S", "bits_w", "bits_s")
 
 def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
                teacher_steps=(1, 2), free_steps: int = 0, warm_check: bool = True,
-               log=print) -> dict:
+               free_chunks: Optional[List[int]] = None, log=print) -> dict:
     """Run wl's warm-up and compressed steps on the GPU (grads regenerated per step on the
     device); check the last warm-up step bit-exactly and the given compressed steps teacher
     forced against the oracle on `chunks` (all chunks when None); run the oracle free-running
@@ -188,8 +190,9 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
                         "warm-up %s differs in chunk %d" % (nm, k)
     opt.freeze()
     free = {}
+    fks = ks if free_chunks is None else [k for k in free_chunks if k in ks]
     if free_steps:
-        for k in ks:
+        for k in fks:
             st = gpu_chunk_state(opt, x, k, ("x", "m", "v"))
             n = st["x"].size
             st["e_w"] = np.zeros((wl.W, n), np.float32)
@@ -201,7 +204,7 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
         wls.torch_fill_grads(wl, g, 1, t)
         tf = t in teacher_steps or (t == last_step and "last" in teacher_steps)
         need_g = tf or t <= free_steps
-        gk = {k: grads_of(k) for k in ks} if need_g else None
+        gk = {k: grads_of(k) for k in (ks if tf else fks)} if need_g else None
         pre = {k: gpu_chunk_state(opt, x, k, PRE) for k in ks} if tf else None
         opt.step(x, g, wl.lr)
         if tf:
@@ -212,7 +215,7 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
                           "inexact_chunks"):
                     stats[f] += getattr(r, f)
         if t <= free_steps:
-            for k in ks:
+            for k in fks:
                 st = free[k]
                 out = oracle.compressed_step(st["x"], st["m"], st["v"], st["e_w"], st["e_s"],
                                              gk[k], wl.C, wl.beta1, wl.eps, wl.lr)
