@@ -178,6 +178,18 @@ def max_over_ranks(value, device):
     return float(t.item())
 
 
+def warmup_phase(wl, warm_ms):
+    """Device time of the full-precision Adam warm-up steps (one launch each): the mean over
+    the steps after the first, and GB/s against their minimum traffic of W*G + 24 bytes per
+    parameter (gradients read; m, v and x read and written)."""
+    if len(warm_ms) < 2:
+        return None
+    ms = sum(warm_ms[1:]) / (len(warm_ms) - 1)
+    nbytes = (wl.W * wl.grad_bytes + 24) * wl.d
+    return {"steps": len(warm_ms), "ms_per_step": ms, "bytes_per_step": nbytes,
+            "achieved_gbs": nbytes / (ms / 1e3) / 1e9}
+
+
 def whole_job_rate(units_per_rank, world, ms_max):
     """Units all ranks processed per second, timed by the slowest rank."""
     return units_per_rank * world / (ms_max / 1e3)
@@ -231,9 +243,16 @@ def run_ours(args):
     x = wls.torch_params(wl, dev)
     g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
     opt = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt, device=dev)
+    warm_ms = []
     for t in range(wl.warmup_steps):             # full-precision Adam warm-up (setup)
         wls.torch_fill_grads(wl, g, 0, t)
+        w0 = torch.cuda.Event(enable_timing=True)
+        w1 = torch.cuda.Event(enable_timing=True)
+        w0.record()
         opt.warmup_step(x, g, wl.lr)
+        w1.record()
+        w1.synchronize()
+        warm_ms.append(w0.elapsed_time(w1))
     opt.freeze()
     wls.torch_fill_grads(wl, g, 1, 1)            # resident inputs for the timed steps
     torch.cuda.synchronize()
@@ -336,6 +355,7 @@ def run_ours(args):
                          "frac": (worker_gbs / peak) if worker_gbs else None,
                          "traffic": ncu_traffic(wl.name),
                          "algorithmic_bytes_per_launch": worker_bytes},
+            "warmup_phase": warmup_phase(wl, warm_ms),
             "gpu_launches": opt.info()["launches_per_step"] * args.steps,
             "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "status_flags": status,
         }

@@ -169,40 +169,97 @@ struct WorkerArgs {
     uint32_t* status;
 };
 
-// 8 resident blocks per SM (at most 32 registers a thread): the kernel is latency-bound on HBM
-// and more warps in flight beat deeper per-thread prefetch (measured on B200).
+// Gradient loads of N consecutive elements (N = 4 or 8): one 16-byte access for 4 fp32 or
+// 8 bf16 values, an 8-byte one for 4 bf16; element by element for a ragged group or when the
+// caller's rows are not 16-byte aligned (VEC false).
+template <typename GT, bool VEC, int N> struct GradLoadN;
+
+template <bool VEC, int N> struct GradLoadN<float, VEC, N> {
+    static __device__ __forceinline__ void load(const float* p, int nv, float (&o)[N]) {
+        if (VEC && nv == N) {
+#pragma unroll
+            for (int h = 0; h < N / 4; ++h) {
+                const float4 t = *reinterpret_cast<const float4*>(p + 4 * h);
+                o[4 * h] = t.x; o[4 * h + 1] = t.y; o[4 * h + 2] = t.z; o[4 * h + 3] = t.w;
+            }
+            return;
+        }
+#pragma unroll
+        for (int c = 0; c < N; ++c) o[c] = c < nv ? p[c] : 0.0f;
+    }
+};
+
+template <bool VEC> struct GradLoadN<uint16_t, VEC, 4> {
+    static __device__ __forceinline__ void load(const uint16_t* p, int nv, float (&o)[4]) {
+        GradLoad<uint16_t, VEC>::load4(p, nv, o);
+    }
+};
+
+template <bool VEC> struct GradLoadN<uint16_t, VEC, 8> {
+    static __device__ __forceinline__ void load(const uint16_t* p, int nv, float (&o)[8]) {
+        if (VEC && nv == 8) {
+            const uint4 t = *reinterpret_cast<const uint4*>(p);
+            const uint32_t u[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                o[2 * h] = __uint_as_float(u[h] << 16);
+                o[2 * h + 1] = __uint_as_float(u[h] & 0xffff0000u);
+            }
+            return;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c) o[c] = c < nv ? __uint_as_float((uint32_t)p[c] << 16) : 0.0f;
+    }
+};
+
+// The kernel is latency-bound on HBM: more warps in flight beat deeper per-thread prefetch
+// (measured on B200). EPT: elements per thread per item, 4 (fp32 gradients: 16-byte loads; 8
+// resident blocks per SM at 32 registers) or 8 (bf16 gradients: 16-byte loads of 8 values; 6
+// blocks per SM at 40 registers, which measured faster than 8 blocks with spills or EPT 4 with
+// 8-byte gradient loads); a 2048-element segment is kSeg / (256 * EPT) items.
 // LAZY_M: the shared momentum is the decompressed server message of the previous step, m =
 // (bit ? S_k : -S_k), rebuilt here from the server plane instead of read as fp32 (4 bytes per
 // parameter fewer to read, and k_apply need not write it).
-template <typename GT, bool VEC, bool LAZY_M>
-__global__ void __launch_bounds__(kThreads, 8) k_worker(const WorkerArgs a) {
+template <typename GT, bool VEC, bool LAZY_M, int EPT>
+__global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const WorkerArgs a) {
+    constexpr int ITEMS = kSeg / (kThreads * EPT);
+    constexpr int LPW = 32 / EPT;  // lanes that share one 32-element sign word
     extern __shared__ double red_w[];  // [W][kWarps]
     int64_t k, j, base, len;
     if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int W = a.geo.W;
+    const int sub = lane & (LPW - 1);
 
-    float mr[kItems][4];
-    int nv[kItems];
+    float mr[ITEMS][EPT];
+    int nv[ITEMS];
 #pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const int64_t off = (int64_t)(it * kThreads + tid) * kVec;
-        nv[it] = valid_of(len, off);
+    for (int it = 0; it < ITEMS; ++it) {
+        const int q = it * kThreads + tid;
+        const int64_t off = (int64_t)q * EPT;
+        const int64_t r = len - off;
+        nv[it] = r <= 0 ? 0 : (r >= EPT ? EPT : (int)r);
         if (nv[it] > 0) {
             if (LAZY_M) {
                 const float S = a.S[k];
-                const uint32_t nib = a.bits_s[(base >> 5) + ((it * kThreads + tid) >> 3)] >> (4 * (lane & 7));
+                const uint32_t bits = a.bits_s[(base >> 5) + q / LPW] >> (EPT * sub);
 #pragma unroll
-                for (int c = 0; c < kVec; ++c) mr[it][c] = ((nib >> c) & 1u) ? S : -S;
+                for (int c = 0; c < EPT; ++c) mr[it][c] = ((bits >> c) & 1u) ? S : -S;
             } else {
-                ld4(a.m + base + off, mr[it]);
+#pragma unroll
+                for (int h = 0; h < EPT / 4; ++h) {
+                    float t4[4];
+                    ld4(a.m + base + off + 4 * h, t4);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) mr[it][4 * h + c] = t4[c];
+                }
             }
         } else {
-            mr[it][0] = mr[it][1] = mr[it][2] = mr[it][3] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) mr[it][c] = 0.0f;
         }
     }
     const float b1 = a.beta1, omb1 = a.omb1;
-    bool nan_seen = false;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
     for (int w = 0; w < W; ++w) {
         const float sp = a.s_lazy[(int64_t)w * a.geo.nch + k];
@@ -211,37 +268,58 @@ __global__ void __launch_bounds__(kThreads, 8) k_worker(const WorkerArgs a) {
         uint32_t* bw = a.bits_w + (int64_t)w * a.geo.ldw + (base >> 5);
         double ss = 0.0;
 #pragma unroll
-        for (int it = 0; it < kItems; ++it) {
+        for (int it = 0; it < ITEMS; ++it) {
             const int q = it * kThreads + tid;
-            const int64_t off = (int64_t)q * kVec;
-            float xp[4] = {0.0f, 0.0f, 0.0f, 0.0f}, gf[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            const int64_t off = (int64_t)q * EPT;
+            float xp[EPT], gf[EPT];
             if (nv[it] > 0) {
-                ld4(ew + off, xp);
-                GradLoad<GT, VEC>::load4(gw + off, nv[it], gf);
-            }
-            float x[4];
-            uint32_t nib = 0u;
 #pragma unroll
-            for (int c = 0; c < kVec; ++c) {
+                for (int h = 0; h < EPT / 4; ++h) {
+                    float t4[4];
+                    ld4(ew + off + 4 * h, t4);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) xp[4 * h + c] = t4[c];
+                }
+                GradLoadN<GT, VEC, EPT>::load(gw + off, nv[it], gf);
+            } else {
+#pragma unroll
+                for (int c = 0; c < EPT; ++c) xp[c] = gf[c] = 0.0f;
+            }
+            float x[EPT];
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) {
                 const float e = __fsub_rn(xp[c], xp[c] >= 0.0f ? sp : -sp);
                 const float mw = __fadd_rn(__fmul_rn(b1, mr[it][c]), __fmul_rn(omb1, gf[c]));
                 const float xv = c < nv[it] ? __fadd_rn(mw, e) : 0.0f;
                 x[c] = xv;
-                nib |= (c < nv[it] && xv >= 0.0f) ? (1u << c) : 0u;
-                nan_seen |= (xv != xv);
-                ss = __fma_rn((double)xv, (double)xv, ss);
+                bits |= (c < nv[it] && xv >= 0.0f) ? (1u << c) : 0u;
+                ss = __fma_rn((double)xv, (double)xv, ss);   // NaN here marks a NaN x_w
             }
-            if (nv[it] > 0) st4(ew + off, x);
-            const uint32_t word = gather_word(nib, lane);
-            if ((lane & 7) == 0 && nv[it] > 0) bw[q >> 3] = word;
+            if (nv[it] > 0) {
+#pragma unroll
+                for (int h = 0; h < EPT / 4; ++h) {
+                    const float t4[4] = {x[4 * h], x[4 * h + 1], x[4 * h + 2], x[4 * h + 3]};
+                    st4(ew + off + 4 * h, t4);
+                }
+            }
+            // OR the LPW lanes' bit groups of one 32-element word together (LSB-first)
+            uint32_t word = bits << (EPT * sub);
+#pragma unroll
+            for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(kFull, word, o);
+            if (sub == 0 && nv[it] > 0) bw[q / LPW] = word;
         }
         ss = warp_sum(ss);
         if (lane == 0) red_w[w * kWarps + warp] = ss;
     }
     __syncthreads();
-    for (int w = tid; w < W; w += kThreads)
-        a.part_w[((int64_t)w * a.geo.nch + k) * a.geo.nseg + j] = block_total(red_w + w * kWarps);
-    if (__syncthreads_or(nan_seen) && tid == 0) atomicOr(a.status, kNanWorker);
+    bool nan_seen = false;
+    for (int w = tid; w < W; w += kThreads) {
+        const double tot = block_total(red_w + w * kWarps);
+        a.part_w[((int64_t)w * a.geo.nch + k) * a.geo.nseg + j] = tot;
+        nan_seen |= (tot != tot);                         // a NaN x_w makes its sum NaN
+    }
+    if (nan_seen) atomicOr(a.status, kNanWorker);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -380,7 +458,7 @@ __host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
 __host__ __device__ inline size_t server_smem_bytes(int W, int nst) {
     const int wpad = (W + 7) & ~7;
     return 64                                                   // mbarriers, mode, unit
-         + (size_t)nst * W * kTileRow * sizeof(uint32_t)        // staged sign words
+         + (size_t)nst * wpad * kTileRow * sizeof(uint32_t)     // staged sign words
          + (size_t)wpad * sizeof(double)                        // scales
          + (size_t)(wpad / 8) * 256 * sizeof(double)            // per-group tables
          + 256 * sizeof(float)                                  // y table (W <= 8)
@@ -454,8 +532,9 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     int* mode_p = reinterpret_cast<int*>(smem_srv + 16);
     int* emin_p = reinterpret_cast<int*>(smem_srv + 20);     // smallest effective exponent
     double* unit_p = reinterpret_cast<double*>(smem_srv + 24);
-    uint32_t* stages = reinterpret_cast<uint32_t*>(smem_srv + 64);      // [nst][W][kTileRow]
-    double* sw = reinterpret_cast<double*>(stages + (size_t)nst * W * kTileRow);
+    // [nst][wpad][kTileRow]; rows W..wpad-1 stay zero, so every group of 8 rows is complete
+    uint32_t* stages = reinterpret_cast<uint32_t*>(smem_srv + 64);
+    double* sw = reinterpret_cast<double*>(stages + (size_t)nst * wpad * kTileRow);
     double* lut = sw + wpad;                                  // fp64 tables [ngroups][256]
     int32_t* ilut = reinterpret_cast<int32_t*>(lut);          // or int32 tables, same place
     float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
@@ -465,10 +544,35 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     if (tid == 0) {
         for (int st = 0; st < nst; ++st) mbar_init(&bars[st], 1);
         for (int t = 0; t < nst && t < nseg_blk; ++t)
-            server_issue(a, stages + (size_t)t * W * kTileRow, &bars[t], c0, clen, j0 + t);
+            server_issue(a, stages + (size_t)t * wpad * kTileRow, &bars[t], c0, clen, j0 + t);
     }
     for (int w = tid; w < wpad; w += kThreads)
         sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
+    for (int st = 0; st < nst; ++st)
+        for (int e = W * kTileRow + tid; e < wpad * kTileRow; e += kThreads)
+            stages[(size_t)st * wpad * kTileRow + e] = 0u;
+    // the first segment's residuals, fetched while the tables are built
+    float zp[kSrvItems][kSrvVec];
+    int nvs[kSrvItems];
+    auto load_residuals = [&](int64_t base, int64_t len) {
+#pragma unroll
+        for (int it = 0; it < kSrvItems; ++it) {
+            const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
+            const int64_t rem = len - off;
+            nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
+            if (nvs[it] > 0) {
+                float h0[4], h1[4];
+                ld4(a.es + base + off, h0);
+                ld4(a.es + base + off + 4, h1);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kSrvVec; ++c) zp[it][c] = 0.0f;
+            }
+        }
+    };
+    load_residuals(c0 + j0 * kSegS, min((int64_t)kSegS, clen - j0 * kSegS));
     __syncthreads();
     if (warp == 0) {
         // exactness bound over the W scales (warp-parallel, fixed reduction order)
@@ -542,7 +646,6 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     const double unit = *unit_p;
     const float Sp = a.S_lazy[k];
     double ss = 0.0;
-    bool nan_seen = false;
 
     for (int t = 0; t < nseg_blk; ++t) {
         const int st = t % nst;
@@ -552,27 +655,10 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
         const int64_t wbase = base >> 5;
         const int lead = (int)(wbase & 3);
         // residuals first, so their latency overlaps the wait for the planes
-        float zp[kSrvItems][kSrvVec];
-        int nvs[kSrvItems];
-#pragma unroll
-        for (int it = 0; it < kSrvItems; ++it) {
-            const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
-            const int64_t rem = len - off;
-            nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
-            if (nvs[it] > 0) {
-                float h0[4], h1[4];
-                ld4(a.es + base + off, h0);
-                ld4(a.es + base + off + 4, h1);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
-            } else {
-#pragma unroll
-                for (int c = 0; c < kSrvVec; ++c) zp[it][c] = 0.0f;
-            }
-        }
+        if (t > 0) load_residuals(base, len);
         const bool landed = mbar_wait_bounded(&bars[st], parity);
         if (landed) {
-            const uint32_t* tile = stages + (size_t)st * W * kTileRow;
+            const uint32_t* tile = stages + (size_t)st * wpad * kTileRow;
 #pragma unroll
             for (int it = 0; it < kSrvItems; ++it) {
                 const int q = it * kThreads + tid;        // 8-element group index in the segment
@@ -584,7 +670,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 if (mode == kModeY) {
                     uint32_t wv[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) wv[i] = (i < W && nv > 0) ? tw[i * kTileRow] : 0u;
+                    for (int i = 0; i < 8; ++i) wv[i] = tw[i * kTileRow];
                     uint32_t lo, hi;
                     gather_bytes(wv, bsel, lo, hi);
                     transpose8x8(lo, hi);
@@ -597,10 +683,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                     for (int g = 0; g < ngroups; ++g) {
                         uint32_t wv[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int w = g * 8 + i;
-                            wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
-                        }
+                        for (int i = 0; i < 8; ++i) wv[i] = tw[(g * 8 + i) * kTileRow];
                         uint32_t lo, hi;
                         gather_bytes(wv, bsel, lo, hi);
                         transpose8x8(lo, hi);
@@ -619,10 +702,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                     for (int g = 0; g < ngroups; ++g) {
                         uint32_t wv[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int w = g * 8 + i;
-                            wv[i] = (w < W && nv > 0) ? tw[w * kTileRow] : 0u;
-                        }
+                        for (int i = 0; i < 8; ++i) wv[i] = tw[(g * 8 + i) * kTileRow];
                         uint32_t lo, hi;
                         gather_bytes(wv, bsel, lo, hi);
                         transpose8x8(lo, hi);
@@ -637,7 +717,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
                     for (int w = 0; w < W; ++w) {
-                        const uint32_t byte = nv > 0 ? (tw[w * kTileRow] >> (8 * bsel)) : 0u;
+                        const uint32_t byte = tw[w * kTileRow] >> (8 * bsel);
                         const double sv = sw[w];
 #pragma unroll
                         for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], ((byte >> c) & 1u) ? sv : -sv);
@@ -653,8 +733,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                     const float zv = c < nv ? __fadd_rn(y[c], e) : 0.0f;
                     z[c] = zv;
                     byte |= (c < nv && zv >= 0.0f) ? (1u << c) : 0u;
-                    nan_seen |= (zv != zv);
-                    ss = __fma_rn((double)zv, (double)zv, ss);
+                    ss = __fma_rn((double)zv, (double)zv, ss);   // NaN here marks a NaN z
                 }
                 if (nv > 0) {
                     const float h0[4] = {z[0], z[1], z[2], z[3]}, h1[4] = {z[4], z[5], z[6], z[7]};
@@ -678,13 +757,16 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             return;
         }
         if (tid == 0 && t + nst < nseg_blk)
-            server_issue(a, stages + (size_t)st * W * kTileRow, &bars[st], c0, clen, j0 + t + nst);
+            server_issue(a, stages + (size_t)st * wpad * kTileRow, &bars[st], c0, clen, j0 + t + nst);
     }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
-    if (tid == 0) a.part_s[k * nsb + b] = block_total(red);
-    if (__syncthreads_or(nan_seen) && tid == 0) atomicOr(a.status, kNanServer);
+    if (tid == 0) {
+        const double tot = block_total(red);
+        a.part_s[k * nsb + b] = tot;
+        if (tot != tot) atomicOr(a.status, kNanServer);   // a NaN z makes the sum NaN
+    }
 }
 
 // ------------------------------------------------------------------------------------------

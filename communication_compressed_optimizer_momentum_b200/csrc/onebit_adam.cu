@@ -135,13 +135,23 @@ int launch_scales(const Geometry& g, const double* part, int64_t rows, int64_t n
     return ONEBIT_OK;
 }
 
+// Vector width of the worker kernel: 8 elements per thread (16-byte loads of 8 bf16 values)
+// when bf16 gradient rows are 16-byte aligned, 4 (16-byte loads of 4 fp32 values, or 8-byte
+// loads of 4 bf16 values) when rows are 16- or 8-byte aligned, element by element otherwise.
 template <typename GT, bool LAZY_M>
 void launch_worker_t(onebit_adam_s* h, const WorkerArgs& a, unsigned blocks, size_t smem,
                      cudaStream_t st) {
-    if (h->geo.d % kVec == 0)
-        k_worker<GT, true, LAZY_M><<<blocks, kThreads, smem, st>>>(a);
+    const int64_t d = h->geo.d;
+    if constexpr (sizeof(GT) == 2) {
+        if (d % 8 == 0) {
+            k_worker<GT, true, LAZY_M, 8><<<blocks, kThreads, smem, st>>>(a);
+            return;
+        }
+    }
+    if (d % kVec == 0)
+        k_worker<GT, true, LAZY_M, 4><<<blocks, kThreads, smem, st>>>(a);
     else
-        k_worker<GT, false, LAZY_M><<<blocks, kThreads, smem, st>>>(a);
+        k_worker<GT, false, LAZY_M, 4><<<blocks, kThreads, smem, st>>>(a);
 }
 
 template <typename GT>
