@@ -28,7 +28,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "worker_kernel_bert_large_bucket.md")
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "step_kernels_bert_large_bucket.md")
 KERNEL_SRC = os.path.join(ROOT, "communication_compressed_optimizer_momentum_b200", "csrc",
                           "kernels.cuh")
 FALLBACK_HBM_GBS = 6650.0
