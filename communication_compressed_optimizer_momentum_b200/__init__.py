@@ -172,6 +172,15 @@ def onebit_last_error() -> str:
     return _abi.lib().onebit_last_error().decode()
 
 
+def onebit_selftest_bounded_wait(polls: int, stream=None) -> bool:
+    """Run the bounded-wait self-test; True when the wait gave up as it should."""
+    import torch
+    flag = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    _check(_abi.lib().onebit_selftest_bounded_wait(polls, _ptr(flag), _stream(stream)),
+           "onebit_selftest_bounded_wait")
+    return int(flag.item()) == 1
+
+
 def onebit_pack(x, words=None, stream=None):
     """Sign-pack a contiguous float32 CUDA tensor into int32 words (LSB-first)."""
     import torch

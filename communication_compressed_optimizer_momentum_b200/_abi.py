@@ -38,6 +38,7 @@ SIGNATURES = {
     "onebit_pack": (INT, [P, I64, P, P]),
     "onebit_unpack": (INT, [P, P, I64, I64, P, P]),
     "onebit_compress_static": (INT, [P, I64, I64, P, P, P]),
+    "onebit_selftest_bounded_wait": (INT, [I32, P, P]),
     "onebit_strerror": (ctypes.c_char_p, [I32]),
     "onebit_last_error": (ctypes.c_char_p, []),
 }

@@ -397,11 +397,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for phase `parity` of the barrier, giving up after kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    for (int i = 0; i < kSpinLimit; ++i)
+// Wait for phase `parity` of the barrier, giving up after `limit` polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  int limit = kSpinLimit) {
+    for (int i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
+}
+
+// Self-test of the bounded wait: arm a barrier for 16 bytes that nothing will deliver and wait
+// on it with the bound the server kernel uses (here `limit` polls). Nothing is copied, so the
+// block can leave with the barrier still pending. *timed_out = 1 when the wait gave up.
+__global__ void k_selftest_wait(int limit, uint32_t* timed_out) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_arrive_expect_tx(&bar, 16);
+    }
+    __syncthreads();
+    const bool landed = mbar_wait_bounded(&bar, 0, limit);
+    const int gave_up = __syncthreads_or(!landed);
+    if (threadIdx.x == 0) *timed_out = gave_up ? 1u : 0u;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -825,41 +841,67 @@ struct WarmupArgs {
     float* x;       // [d] caller-owned
 };
 
-template <typename GT, bool VEC>
-__global__ void __launch_bounds__(kThreads) k_warmup(const WarmupArgs a) {
+// EPT elements per thread as in k_worker (8 for bf16, 4 for fp32 gradients). The fp64 sum over
+// workers runs in worker order (bit-exact with the definition); the gradient loads of UNR
+// workers are issued together so that they are in flight at once.
+template <typename GT, bool VEC, int EPT>
+__global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
+    constexpr int ITEMS = kSeg / (kThreads * EPT);
+    constexpr int UNR = 4;
     int64_t k, j, base, len;
     if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x;
+    const int W = a.geo.W;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
-    const double dW = (double)a.geo.W;
+    const double dW = (double)W;
 #pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const int64_t off = (int64_t)(it * kThreads + tid) * kVec;
-        const int nv = valid_of(len, off);
+    for (int it = 0; it < ITEMS; ++it) {
+        const int64_t off = (int64_t)(it * kThreads + tid) * EPT;
+        const int64_t r = len - off;
+        const int nv = r <= 0 ? 0 : (r >= EPT ? EPT : (int)r);
         if (nv == 0) continue;
-        double acc[4] = {0.0, 0.0, 0.0, 0.0};
-        for (int w = 0; w < a.geo.W; ++w) {
-            float gf[4];
-            GradLoad<GT, VEC>::load4(g0 + (int64_t)w * a.geo.d + off, nv, gf);
+        double acc[EPT];
 #pragma unroll
-            for (int c = 0; c < kVec; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[c]);
-        }
-        float m[4], v[4], x[4];
-        ld4(a.m + base + off, m);
-        ld4(a.v + base + off, v);
-        ld4_caller(a.x + base + off, nv, x);
+        for (int c = 0; c < EPT; ++c) acc[c] = 0.0;
+        int w = 0;
+        for (; w + UNR <= W; w += UNR) {
+            float gf[UNR][EPT];
 #pragma unroll
-        for (int c = 0; c < kVec; ++c) {
-            if (c >= nv) continue;
-            const float gbar = __double2float_rn(__ddiv_rn(acc[c], dW));
-            m[c] = __fadd_rn(__fmul_rn(a.beta1, m[c]), __fmul_rn(a.omb1, gbar));
-            v[c] = __fadd_rn(__fmul_rn(a.beta2, v[c]), __fmul_rn(a.omb2, __fmul_rn(gbar, gbar)));
-            const float den = __fadd_rn(__fsqrt_rn(v[c]), a.eps);
-            x[c] = __fsub_rn(x[c], __fmul_rn(a.lr, __fdiv_rn(m[c], den)));
+            for (int u = 0; u < UNR; ++u)
+                GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)(w + u) * a.geo.d + off, nv, gf[u]);
+#pragma unroll
+            for (int u = 0; u < UNR; ++u)
+#pragma unroll
+                for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[u][c]);
         }
-        st4(a.m + base + off, m);
-        st4(a.v + base + off, v);
-        st4_caller(a.x + base + off, nv, x);
+        for (; w < W; ++w) {
+            float gf[EPT];
+            GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)w * a.geo.d + off, nv, gf);
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[c]);
+        }
+#pragma unroll
+        for (int h = 0; h < EPT / 4; ++h) {
+            const int64_t o4 = off + 4 * h;
+            const int nv4 = nv - 4 * h;
+            if (nv4 <= 0) break;
+            float m[4], v[4], x[4];
+            ld4(a.m + base + o4, m);
+            ld4(a.v + base + o4, v);
+            ld4_caller(a.x + base + o4, nv4 >= 4 ? 4 : nv4, x);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c >= nv4) continue;
+                const float gbar = __double2float_rn(__ddiv_rn(acc[4 * h + c], dW));
+                m[c] = __fadd_rn(__fmul_rn(a.beta1, m[c]), __fmul_rn(a.omb1, gbar));
+                v[c] = __fadd_rn(__fmul_rn(a.beta2, v[c]), __fmul_rn(a.omb2, __fmul_rn(gbar, gbar)));
+                const float den = __fadd_rn(__fsqrt_rn(v[c]), a.eps);
+                x[c] = __fsub_rn(x[c], __fmul_rn(a.lr, __fdiv_rn(m[c], den)));
+            }
+            st4(a.m + base + o4, m);
+            st4(a.v + base + o4, v);
+            st4_caller(a.x + base + o4, nv4 >= 4 ? 4 : nv4, x);
+        }
     }
 }
 

@@ -183,10 +183,18 @@ int launch_warmup(onebit_adam_s* h, float* x, const void* grads, float lr, cudaS
     WarmupArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->beta2, 1.0f - h->beta2, h->eps, lr,
                  grads, h->m, h->v, x};
     const unsigned blocks = (unsigned)step_blocks(h->geo);
-    if (h->geo.d % kVec == 0)
-        k_warmup<GT, true><<<blocks, kThreads, 0, st>>>(a);
+    const int64_t d = h->geo.d;
+    if constexpr (sizeof(GT) == 2) {
+        if (d % 8 == 0) {
+            k_warmup<GT, true, 8><<<blocks, kThreads, 0, st>>>(a);
+            ONEBIT_CUDA(cudaGetLastError());
+            return ONEBIT_OK;
+        }
+    }
+    if (d % kVec == 0)
+        k_warmup<GT, true, 4><<<blocks, kThreads, 0, st>>>(a);
     else
-        k_warmup<GT, false><<<blocks, kThreads, 0, st>>>(a);
+        k_warmup<GT, false, 4><<<blocks, kThreads, 0, st>>>(a);
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }
@@ -603,6 +611,14 @@ void onebit_adam_destroy(onebit_adam_t h) {
     if (h == nullptr) return;
     free_events(h);
     delete h;
+}
+
+int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* stream) {
+    if (polls < 1 || polls > kSpinLimit || timed_out == nullptr) return ONEBIT_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(timed_out) & 3u) return ONEBIT_ERR_ALIGN;
+    k_selftest_wait<<<1, 32, 0, as_stream(stream)>>>(polls, timed_out);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
 }
 
 int onebit_pack(const float* x, int64_t n, uint32_t* words, void* stream) {

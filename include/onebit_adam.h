@@ -225,6 +225,16 @@ int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t
 int onebit_compress_static(const float* x, int64_t n, int64_t C, uint32_t* words, float* scales,
                            void* stream);
 
+/*
+ * Self-test of failure detection without a GPU fault: one block arms an mbarrier for bytes
+ * that never arrive and waits on it with the same bounded wait the server kernel uses, giving
+ * up after `polls` polls (1 <= polls <= 2^22). Writes 1 to *timed_out (device, 4-byte aligned)
+ * when the wait gave up -- the expected outcome -- and 0 if it did not. The kernel returns
+ * normally and the context stays usable. No counterpart in the paper; this is library
+ * plumbing for the bounded waits.
+ */
+int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* stream);
+
 /* Static description of a status code. */
 const char* onebit_strerror(int32_t code);
 

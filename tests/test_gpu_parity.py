@@ -285,3 +285,40 @@ def test_timing_reports_each_kernel():
     assert all(v > 0 for v in ms.values()), ms
     opt.timing(0)
     opt.close()
+
+
+def test_bounded_wait_gives_up_and_the_context_survives():
+    """Failure detection without a GPU fault: a wait on bytes that never arrive expires after
+    its bound, the kernel returns, and the device keeps working."""
+    assert ob.onebit_selftest_bounded_wait(1000)
+    assert ob.onebit_selftest_bounded_wait(20_000)
+    x = torch.ones(4096, device=DEV)
+    words = ob.onebit_pack(x)
+    torch.cuda.synchronize()
+    assert int(words[0].item()) == -1          # all 32 signs positive
+
+
+def test_bench_json_line_contract(tmp_path):
+    """bench.py prints one JSON line with the keys the benchmark contract names."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--workload", "smoke_1m",
+                        "--steps", "3", "--warmup", "3", "--e2e-steps", "1",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "cpu_baseline", "e2e", "clocks", "gpu_launches"):
+        assert key in j, key
+    assert j["value"] > 0 and j["steps"] == 3 and j["n_gpus"] == 1
+    assert j["config"]["workload"] == "smoke_1m"
+    assert j["gpu_launches"] == 15
+    roof = j["roofline"]
+    assert roof["bound"] == "hbm" and roof["unit"] == "GB/s" and roof["peak"] > 0
+    assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
+    assert j["e2e"]["h2d_bytes_per_step"] == 4 * 1_048_576 * 4
+    assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
