@@ -5,10 +5,11 @@
 // flight. The work unit is a SEGMENT of consecutive elements that never crosses a chunk
 // boundary (chunk k = elements [kC, kC + C_k), LIT-278 note, Key takeaways: per-chunk scaling):
 // kSeg = 2048 elements for the worker, apply and warm-up kernels, kSegS = 4096 for the server
-// kernel. A block owns one segment; in the 2048-element kernels thread t owns kItems groups of
-// kVec = 4 consecutive elements at offsets (it * kThreads + t) * 4, so each warp-wide access is
-// one contiguous 512-byte run. Small per-thread state (about 40 registers) keeps 48 warps per SM
-// in flight, which is what hides HBM latency here.
+// kernel. A block owns one segment (the server kernel a run of up to 8 segments of one chunk);
+// thread t owns groups of 4 or 8 consecutive elements at offsets (it * kThreads + t) * EPT, so
+// each warp-wide access is one contiguous 512- or 1024-byte run of 16-byte accesses. Small
+// per-thread state (32-40 registers) keeps 48-64 warps per SM in flight, which is what hides
+// HBM latency here.
 //
 // Determinism: chunk norms are fp64 sums in a fixed tree (thread -> warp butterfly -> block in
 // warp order -> segments in order), so a run is bit-reproducible; no float atomics anywhere.
@@ -104,32 +105,6 @@ __device__ __forceinline__ void st4_caller(float* p, int nv, const float (&o)[4]
         if (c < nv) p[c] = o[c];
 }
 
-// Gradient element types: fp32, or bf16 bit patterns (uint16_t) that widen exactly.
-template <typename GT, bool VEC> struct GradLoad;
-
-template <bool VEC> struct GradLoad<float, VEC> {
-    static __device__ __forceinline__ void load4(const float* p, int nv, float (&o)[4]) {
-        if (VEC && nv == kVec) { ld4(p, o); return; }
-#pragma unroll
-        for (int c = 0; c < kVec; ++c) o[c] = c < nv ? p[c] : 0.0f;
-    }
-};
-
-template <bool VEC> struct GradLoad<uint16_t, VEC> {
-    static __device__ __forceinline__ void load4(const uint16_t* p, int nv, float (&o)[4]) {
-        if (VEC && nv == kVec) {
-            const uint2 t = *reinterpret_cast<const uint2*>(p);
-            o[0] = __uint_as_float(t.x << 16);
-            o[1] = __uint_as_float(t.x & 0xffff0000u);
-            o[2] = __uint_as_float(t.y << 16);
-            o[3] = __uint_as_float(t.y & 0xffff0000u);
-            return;
-        }
-#pragma unroll
-        for (int c = 0; c < kVec; ++c) o[c] = c < nv ? __uint_as_float((uint32_t)p[c] << 16) : 0.0f;
-    }
-};
-
 // OR together the nibbles of the 8 lanes that share one 32-element word; lane l contributes
 // elements 4(l%8)..4(l%8)+3 of the word (LSB-first).
 __device__ __forceinline__ uint32_t gather_word(uint32_t nib, int lane) {
@@ -169,9 +144,10 @@ struct WorkerArgs {
     uint32_t* status;
 };
 
-// Gradient loads of N consecutive elements (N = 4 or 8): one 16-byte access for 4 fp32 or
-// 8 bf16 values, an 8-byte one for 4 bf16; element by element for a ragged group or when the
-// caller's rows are not 16-byte aligned (VEC false).
+// Gradient loads of N consecutive elements (N = 4 or 8), fp32 or bf16 bit patterns (uint16_t,
+// widened exactly by a 16-bit shift): one 16-byte access for 4 fp32 or 8 bf16 values, an 8-byte
+// one for 4 bf16; element by element for a ragged group or when the caller's rows are not
+// aligned for vector access (VEC false).
 template <typename GT, bool VEC, int N> struct GradLoadN;
 
 template <bool VEC, int N> struct GradLoadN<float, VEC, N> {
@@ -191,7 +167,16 @@ template <bool VEC, int N> struct GradLoadN<float, VEC, N> {
 
 template <bool VEC> struct GradLoadN<uint16_t, VEC, 4> {
     static __device__ __forceinline__ void load(const uint16_t* p, int nv, float (&o)[4]) {
-        GradLoad<uint16_t, VEC>::load4(p, nv, o);
+        if (VEC && nv == 4) {
+            const uint2 t = *reinterpret_cast<const uint2*>(p);
+            o[0] = __uint_as_float(t.x << 16);
+            o[1] = __uint_as_float(t.x & 0xffff0000u);
+            o[2] = __uint_as_float(t.y << 16);
+            o[3] = __uint_as_float(t.y & 0xffff0000u);
+            return;
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) o[c] = c < nv ? __uint_as_float((uint32_t)p[c] << 16) : 0.0f;
     }
 };
 
@@ -460,7 +445,7 @@ struct ServerArgs {
     float* es;               // [ld] lazy server residual: holds last step's z
     const float* S_lazy;     // [nch]
     uint32_t* bits_s;        // [ldw]
-    double* part_s;          // [nch][nseg_s]
+    double* part_s;          // [nch][blocks per chunk]: one fp64 partial per block
     uint32_t* status;
 };
 

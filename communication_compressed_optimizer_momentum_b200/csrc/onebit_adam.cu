@@ -19,6 +19,7 @@
 #include <vector>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>  // header-only; ranges are free unless a profiler is attached
 
 #include "onebit_adam.h"
 #include "kernels.cuh"
@@ -360,6 +361,11 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
     const Geometry& g = h->geo;
     const unsigned blocks = (unsigned)step_blocks(g);
     int rc;
+    // one profiler range per step (NVTX; a no-op without a tool attached)
+    struct Range {
+        Range() { nvtxRangePushA("onebit_adam_compressed_step"); }
+        ~Range() { nvtxRangePop(); }
+    } range;
 
     record(h, 0, st);
     rc = h->gtype == ONEBIT_BF16 ? launch_worker<uint16_t>(h, grads, st)
