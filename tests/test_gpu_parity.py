@@ -322,3 +322,40 @@ def test_bench_json_line_contract(tmp_path):
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
     assert j["e2e"]["h2d_bytes_per_step"] == 4 * 1_048_576 * 4
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+
+
+def test_cuda_graph_replay_matches_eager():
+    """A compressed step queues kernels only (no host synchronisation), so it can be captured
+    in a CUDA graph. After the first step (which reads the explicit warm-up momentum) every step
+    launches the same kernels, so replays of a captured step equal eager steps bit for bit."""
+    d, W, C = 200_000, 4, 16_384
+    gl = _grads(W, d, 6, 5)
+    g_static = torch.empty_like(gl[0])
+    xa = torch.linspace(-0.05, 0.05, d, device=DEV)
+    xb = xa.clone()
+    a = ob.OneBitAdam(d, W, C, device=DEV)
+    b = ob.OneBitAdam(d, W, C, device=DEV)
+    for o in (a, b):
+        o.freeze()
+    a.step(xa, gl[0], 1e-3)
+    b.step(xb, gl[0], 1e-3)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    g_static.copy_(gl[1])
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=s):
+        b.step(xb, g_static, 1e-3)
+    # capture records the launches without running them: replay once per step from here on
+    for g in gl[1:]:
+        a.step(xa, g, 1e-3)
+        g_static.copy_(g)
+        graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(xa, xb)
+    for k in ("m", "e_w", "e_s", "bits_s"):
+        assert torch.equal(a.get_state(k), b.get_state(k)), k
+    del graph
+    a.close()
+    b.close()
