@@ -224,7 +224,6 @@ def oracle_sample_rate(wl, state, g, seconds):
 
 
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -388,7 +387,6 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    import numpy as np
     import oracle
     from communication_compressed_optimizer_momentum_b200 import workloads as wls
     wl = get_workload(args.workload)

@@ -11,7 +11,7 @@ raised.
 from __future__ import annotations
 
 import ctypes
-from typing import Optional, Tuple
+from typing import Tuple
 
 from . import _abi
 

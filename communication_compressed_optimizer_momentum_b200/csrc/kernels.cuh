@@ -813,6 +813,19 @@ __global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
     }
 }
 
+
+// bf16 bit pattern -> the exactly equal fp64 value. Normal values and +-0 by integer ops (the
+// 8-bit exponent rebiased to 11 bits, the 7-bit fraction moved up); subnormal, inf and NaN
+// inputs through the fp32 conversion.
+__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
+    const uint32_t mag = b & 0x7fffu, e = mag >> 7;
+    if (e == 0u || e == 0xffu) {
+        if (mag == 0u) return __hiloint2double((int)((b & 0x8000u) << 16), 0);
+        return (double)__uint_as_float(b << 16);
+    }
+    return __hiloint2double((int)(((b & 0x8000u) << 16) | ((mag << 13) + 0x38000000u)), 0);
+}
+
 // ------------------------------------------------------------------------------------------
 // Warm-up: one full-precision Adam step on the fp64 worker average (LIT-278 note, "What the
 // evidence does not cover": the warm-up phase is plain Adam). No bias correction.
@@ -849,6 +862,23 @@ __global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
 #pragma unroll
         for (int c = 0; c < EPT; ++c) acc[c] = 0.0;
         int w = 0;
+        if constexpr (sizeof(GT) == 2 && VEC && EPT == 8) {
+            for (; w + UNR <= W && nv == EPT; w += UNR) {
+                uint4 raw[UNR];
+#pragma unroll
+                for (int u = 0; u < UNR; ++u)
+                    raw[u] = *reinterpret_cast<const uint4*>(g0 + (int64_t)(w + u) * a.geo.d + off);
+#pragma unroll
+                for (int u = 0; u < UNR; ++u) {
+                    const uint32_t r[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        acc[2 * h] = __dadd_rn(acc[2 * h], bf16_to_f64(r[h] & 0xffffu));
+                        acc[2 * h + 1] = __dadd_rn(acc[2 * h + 1], bf16_to_f64(r[h] >> 16));
+                    }
+                }
+            }
+        }
         for (; w + UNR <= W; w += UNR) {
             float gf[UNR][EPT];
 #pragma unroll

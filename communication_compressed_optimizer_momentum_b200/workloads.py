@@ -15,8 +15,7 @@ parity always hands the oracle the exact bytes the device consumed.
 from __future__ import annotations
 
 import dataclasses
-import math
-from typing import List, Optional, Sequence, Tuple
+from typing import List, Optional, Tuple
 
 import numpy as np
 

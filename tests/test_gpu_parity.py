@@ -13,7 +13,7 @@ import torch
 import communication_compressed_optimizer_momentum_b200 as ob
 import oracle
 from communication_compressed_optimizer_momentum_b200 import workloads as wls
-from gpu_helpers import DEV, padding_is_zero, run_parity, to_np, unpack_bits
+from gpu_helpers import DEV, padding_is_zero, run_parity, to_np
 
 pytestmark = pytest.mark.gpu
 
