@@ -1,0 +1,106 @@
+"""Host-side logic without a GPU: workload shapes, the benchmark's parsing of the committed ncu
+summary and of nvidia-smi samples, and its derived figures."""
+import hashlib
+import json
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from communication_compressed_optimizer_momentum_b200 import workloads as wls  # noqa: E402
+
+
+def test_bucket_shapes_are_the_sums_of_their_tensors():
+    assert wls.transformer_layer_params(768, 3072) == 7_087_872
+    assert wls.WORKLOADS["bert_base_bucket"].d == 12 * 7_087_872 + 30522 * 768 == 108_495_360
+    assert wls.WORKLOADS["bert_large_bucket"].d == 24 * 12_596_224 + 30522 * 1024 == 333_563_904
+    assert wls.WORKLOADS["gpt2_xl_bucket"].d == 48 * 30_740_800 + 50257 * 1600 == 1_555_969_600
+    bl = wls.WORKLOADS["bert_large_bucket"]
+    assert bl.C * bl.W == bl.d and bl.nch == 16
+    g2 = wls.WORKLOADS["gpt2_xl_bucket"]
+    assert g2.nch == 371 and g2.d - 370 * g2.C == 4_077_120
+    for w in wls.WORKLOADS.values():
+        assert w.d % 32 == 0 and w.C % 32 == 0
+        assert sum(w.layer_sizes or (w.d,)) == w.d
+
+
+def test_sweep_points_and_chunk_rounding():
+    pts = wls.sweep_points()
+    assert len(pts) == 24
+    for W, C in pts:
+        wl = wls.sweep_workload(W, C)
+        assert wl.C % 32 == 0 and wl.d == 1 << 28
+        if C is None:
+            assert wl.C * W >= wl.d and (wl.C - 32) * W < wl.d
+
+
+def test_algorithmic_bytes_split_by_kernel():
+    for w in list(wls.WORKLOADS.values()) + [wls.sweep_workload(64, None)]:
+        kb = w.kernel_bytes_per_param()
+        assert sum(kb.values()) == pytest.approx(w.algorithmic_bytes_per_param())
+    assert wls.WORKLOADS["bert_large_bucket"].algorithmic_bytes_per_param() == 184.375
+
+
+def test_scaled_workload_keeps_segment_proportions():
+    wl = wls.scaled(wls.WORKLOADS["bert_base_bucket"], 1 << 20)
+    assert wl.d == 1 << 20 and sum(wl.layer_sizes) == wl.d and len(wl.layer_sizes) == 13
+
+
+def test_host_generators_are_seeded_and_shaped():
+    wl = wls.scaled(wls.WORKLOADS["bert_large_bucket"], 4096)
+    a, b = wls.np_grads(wl, 1, 3), wls.np_grads(wl, 1, 3)
+    assert a.dtype == np.uint16 and a.shape == (wl.W, 4096) and np.array_equal(a, b)
+    assert not np.array_equal(a, wls.np_grads(wl, 1, 4))
+    f = wls.bf16_bits_to_f32(a)
+    assert np.isfinite(f).all() and 1e-4 < float(np.std(f)) < 1e-1
+
+
+def test_ncu_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    sha = bench.kernel_source_sha()
+    p = tmp_path / "summary.md"
+    p.write_text("- workload: `bert_large_bucket`\n- kernel_source_sha256: `%s`\n"
+                 "- dram_bytes_per_launch_full: `123456`\n" % sha)
+    monkeypatch.setattr(bench, "PROFILE_SUMMARY", str(p))
+    assert bench.ncu_traffic("bert_large_bucket") == 123456.0
+    assert bench.ncu_traffic("smoke_1m") is None              # other workload
+    p.write_text(p.read_text().replace(sha, "0" * 64))
+    assert bench.ncu_traffic("bert_large_bucket") is None      # stale: kernels changed since
+
+
+def test_committed_profile_summary_parses():
+    with open(bench.PROFILE_SUMMARY) as f:
+        text = f.read()
+    assert "kernel_source_sha256" in text and "dram_bytes_per_launch_full" in text
+
+
+def test_warmup_phase_figures():
+    wl = wls.WORKLOADS["bert_large_bucket"]
+    r = bench.warmup_phase(wl, [9.0, 4.0, 4.0])
+    assert r["ms_per_step"] == 4.0 and r["bytes_per_step"] == (16 * 2 + 24) * wl.d
+    assert r["achieved_gbs"] == pytest.approx(r["bytes_per_step"] / 4e-3 / 1e9)
+    assert bench.warmup_phase(wl, [1.0]) is None
+
+
+def test_clock_sampler_parses_nvidia_smi_lines():
+    s = bench.ClockSampler(0)
+    s.proc = type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout: 0})()
+    s.t0, s.t1 = 100.0, 101.0
+    s.lines = [(100.1, "2026/12/02 17:00:00.000, 0, 1650, 1965, 980.5, 0x4, Not Active, "
+                       "Not Active, Not Active, Active"),
+               (100.5, "2026/12/02 17:00:00.200, 0, 1700, 1965, 990.0, 0x0, Not Active, "
+                       "Not Active, Not Active, Not Active"),
+               (150.0, "2026/12/02 17:00:50.000, 0, 120, 1965, 90.0, 0x0, Not Active, "
+                       "Not Active, Not Active, Not Active")]
+    c = s.stop()
+    assert c["samples"] == 2 and c["in_timed_region"]
+    assert c["sm_mhz"] in (1650.0, 1700.0) and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+
+
+def test_whole_job_rate():
+    assert bench.whole_job_rate(1000, 4, 2.0) == pytest.approx(4000 / 0.002)
