@@ -455,11 +455,20 @@ __host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
     return (W <= 128 && nseg_s > 1) ? 2 : 1;
 }
 
+// Residuals staged by TMA next to the sign words (STAGE_RES) while the stages stay small enough
+// for several blocks per SM; for wider W they are read into registers instead (measured).
+__host__ __device__ inline bool server_stage_residuals(int W) { return W <= 32; }
+
+// Words of one pipeline stage: wpad plane rows, then the segment's residuals when staged.
+__host__ __device__ inline size_t server_stage_words(int W, bool stage_res) {
+    return (size_t)((W + 7) & ~7) * kTileRow + (stage_res ? kSegS : 0);
+}
+
 // Dynamic shared memory of k_server for W workers and `nst` stages (bytes).
 __host__ __device__ inline size_t server_smem_bytes(int W, int nst) {
     const int wpad = (W + 7) & ~7;
     return 64                                                   // mbarriers, mode, unit
-         + (size_t)nst * wpad * kTileRow * sizeof(uint32_t)     // staged sign words
+         + (size_t)nst * server_stage_words(W, server_stage_residuals(W)) * sizeof(uint32_t)
          + (size_t)wpad * sizeof(double)                        // scales
          + (size_t)(wpad / 8) * 256 * sizeof(double)            // per-group tables
          + 256 * sizeof(float)                                  // y table (W <= 8)
@@ -496,8 +505,10 @@ __device__ __forceinline__ float server_average(double acc, double dW, double in
     return __double2float_rn(POW2 ? acc * invW : __ddiv_rn(acc, dW));
 }
 
-// Start the bulk copies of segment j's W plane rows into one stage (thread 0 only).
-__device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stage,
+// Start the bulk copies of segment j's W plane rows -- and, with STAGE_RES, its residuals after
+// the wpad rows -- into one stage (thread 0 only).
+template <bool STAGE_RES>
+__device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stage, int wpad,
                                              uint64_t* bar, int64_t c0, int64_t clen,
                                              int64_t j) {
     const int64_t base = c0 + j * kSegS;
@@ -507,13 +518,17 @@ __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stag
     // aligned and inside the row (plane rows are padded to a multiple of 4 words)
     const int lead = (int)(wbase & 3);
     const uint32_t row_bytes = (uint32_t)(((lead + (len + 31) / 32 + 3) / 4) * 16);
-    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)a.geo.W);
+    // residuals [base, base + round_up(len, 4)): base is a multiple of 32 elements and the
+    // buffer is padded to a multiple of 64, so the copy is 16-byte aligned and in bounds
+    const uint32_t es_bytes = STAGE_RES ? (uint32_t)(((len + 3) / 4) * 16) : 0u;
+    mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)a.geo.W + es_bytes);
     for (int w = 0; w < a.geo.W; ++w)
         bulk_load(stage + (size_t)w * kTileRow,
                   a.bits_w + (int64_t)w * a.geo.ldw + (wbase - lead), row_bytes, bar);
+    if (STAGE_RES) bulk_load(stage + (size_t)wpad * kTileRow, a.es + base, es_bytes, bar);
 }
 
-template <bool POW2>
+template <bool POW2, bool STAGE_RES>
 __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     extern __shared__ __align__(16) unsigned char smem_srv[];
     const int W = a.geo.W;
@@ -533,9 +548,11 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     int* mode_p = reinterpret_cast<int*>(smem_srv + 16);
     int* emin_p = reinterpret_cast<int*>(smem_srv + 20);     // smallest effective exponent
     double* unit_p = reinterpret_cast<double*>(smem_srv + 24);
-    // [nst][wpad][kTileRow]; rows W..wpad-1 stay zero, so every group of 8 rows is complete
+    // [nst][stage_words]: wpad plane rows (rows W..wpad-1 stay zero, so every group of 8 rows
+    // is complete), then, with STAGE_RES, the segment's residuals
+    const size_t stage_words = server_stage_words(W, STAGE_RES);
     uint32_t* stages = reinterpret_cast<uint32_t*>(smem_srv + 64);
-    double* sw = reinterpret_cast<double*>(stages + (size_t)nst * wpad * kTileRow);
+    double* sw = reinterpret_cast<double*>(stages + (size_t)nst * stage_words);
     double* lut = sw + wpad;                                  // fp64 tables [ngroups][256]
     int32_t* ilut = reinterpret_cast<int32_t*>(lut);          // or int32 tables, same place
     float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
@@ -545,14 +562,15 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     if (tid == 0) {
         for (int st = 0; st < nst; ++st) mbar_init(&bars[st], 1);
         for (int t = 0; t < nst && t < nseg_blk; ++t)
-            server_issue(a, stages + (size_t)t * wpad * kTileRow, &bars[t], c0, clen, j0 + t);
+            server_issue<STAGE_RES>(a, stages + (size_t)t * stage_words, wpad, &bars[t], c0, clen,
+                                    j0 + t);
     }
     for (int w = tid; w < wpad; w += kThreads)
         sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
     for (int st = 0; st < nst; ++st)
         for (int e = W * kTileRow + tid; e < wpad * kTileRow; e += kThreads)
-            stages[(size_t)st * wpad * kTileRow + e] = 0u;
-    // the first segment's residuals, fetched while the tables are built
+            stages[(size_t)st * stage_words + e] = 0u;
+    // without STAGE_RES: the first segment's residuals, fetched while the tables are built
     float zp[kSrvItems][kSrvVec];
     int nvs[kSrvItems];
     auto load_residuals = [&](int64_t base, int64_t len) {
@@ -573,7 +591,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             }
         }
     };
-    load_residuals(c0 + j0 * kSegS, min((int64_t)kSegS, clen - j0 * kSegS));
+    if (!STAGE_RES) load_residuals(c0 + j0 * kSegS, min((int64_t)kSegS, clen - j0 * kSegS));
     __syncthreads();
     if (warp == 0) {
         // exactness bound over the W scales (warp-parallel, fixed reduction order)
@@ -656,10 +674,24 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
         const int64_t wbase = base >> 5;
         const int lead = (int)(wbase & 3);
         // residuals first, so their latency overlaps the wait for the planes
-        if (t > 0) load_residuals(base, len);
+        if (!STAGE_RES && t > 0) load_residuals(base, len);
         const bool landed = mbar_wait_bounded(&bars[st], parity);
         if (landed) {
-            const uint32_t* tile = stages + (size_t)st * wpad * kTileRow;
+            const uint32_t* tile = stages + (size_t)st * stage_words;
+            if (STAGE_RES) {
+                const float* res = reinterpret_cast<const float*>(tile + (size_t)wpad * kTileRow);
+#pragma unroll
+                for (int it = 0; it < kSrvItems; ++it) {
+                    const int64_t off = (int64_t)(it * kThreads + tid) * kSrvVec;
+                    const int64_t rem = len - off;
+                    nvs[it] = rem <= 0 ? 0 : (rem >= kSrvVec ? kSrvVec : (int)rem);
+                    float h0[4], h1[4];
+                    ld4(res + off, h0);
+                    ld4(res + off + 4, h1);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) { zp[it][c] = h0[c]; zp[it][c + 4] = h1[c]; }
+                }
+            }
 #pragma unroll
             for (int it = 0; it < kSrvItems; ++it) {
                 const int q = it * kThreads + tid;        // 8-element group index in the segment
@@ -758,7 +790,8 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             return;
         }
         if (tid == 0 && t + nst < nseg_blk)
-            server_issue(a, stages + (size_t)st * wpad * kTileRow, &bars[st], c0, clen, j0 + t + nst);
+            server_issue<STAGE_RES>(a, stages + (size_t)st * stage_words, wpad, &bars[st], c0,
+                                    clen, j0 + t + nst);
     }
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;

@@ -117,6 +117,15 @@ int64_t server_blocks_per_chunk(const Geometry& g) {
 }
 int64_t server_blocks(const Geometry& g) { return g.nch * server_blocks_per_chunk(g); }
 
+// The k_server instantiation for W workers: exact scaling for power-of-two W, residuals staged
+// by TMA for narrow W.
+using ServerKernel = void (*)(ServerArgs);
+ServerKernel server_kernel(int W) {
+    const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W);
+    if (pow2) return staged ? k_server<true, true> : k_server<true, false>;
+    return staged ? k_server<false, true> : k_server<false, false>;
+}
+
 // Launch the chunk-scale reduction (nseg partials of seg elements per row) with the thread
 // count that fits the partial count.
 int launch_scales(const Geometry& g, const double* part, int64_t rows, int64_t nseg, int seg,
@@ -312,8 +321,8 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->status = reinterpret_cast<uint32_t*>(b + L.status);
     h->gtype = grad_dtype;
     const int ssm = (int)server_smem_bytes(h->geo.W, server_stages(h->geo.W, h->geo.nseg_s));
-    ONEBIT_CUDA(cudaFuncSetAttribute(k_server<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
-    ONEBIT_CUDA(cudaFuncSetAttribute(k_server<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
+    ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel(h->geo.W),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     cudaStream_t st = as_stream(stream);
     // m and v start at zero (Adam); the rest is cleared too so padding is deterministic.
     ONEBIT_CUDA(cudaMemsetAsync(b, 0, L.total, st));
@@ -378,10 +387,7 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
     ServerArgs sa{g, h->bits_w, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s, h->status};
     const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
     const unsigned sblocks = (unsigned)server_blocks(g);
-    if ((g.W & (g.W - 1)) == 0)
-        k_server<true><<<sblocks, kThreads, ssm, st>>>(sa);
-    else
-        k_server<false><<<sblocks, kThreads, ssm, st>>>(sa);
+    server_kernel(g.W)<<<sblocks, kThreads, ssm, st>>>(sa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 3, st);
     rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
