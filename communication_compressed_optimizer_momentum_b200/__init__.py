@@ -111,6 +111,10 @@ def onebit_adam_compressed_step_host(h, x_dev, grads_dev, grads_host, x_host, lr
         _stream(stream)), "onebit_adam_compressed_step_host")
 
 
+def onebit_adam_host_wait(h, stream=None) -> None:
+    _check(_abi.lib().onebit_adam_host_wait(_handle(h), _stream(stream)), "onebit_adam_host_wait")
+
+
 def onebit_adam_state_bytes(h, which: int) -> int:
     n = ctypes.c_uint64()
     _check(_abi.lib().onebit_adam_state_bytes(_handle(h), which, ctypes.byref(n)),
@@ -254,6 +258,9 @@ class OneBitAdam:
 
     def step_host(self, x_dev, grads_dev, grads_host, x_host, lr: float, stream=None) -> None:
         onebit_adam_compressed_step_host(self.h, x_dev, grads_dev, grads_host, x_host, lr, stream)
+
+    def host_wait(self, stream=None) -> None:
+        onebit_adam_host_wait(self.h, stream)
 
     def state_shape(self, which: str):
         d, W, nch, nw = self.d, self.W, self.nch, (self.d + 31) // 32

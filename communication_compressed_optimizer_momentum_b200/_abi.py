@@ -26,6 +26,7 @@ SIGNATURES = {
     "onebit_adam_freeze_variance": (INT, [P, P]),
     "onebit_adam_compressed_step": (INT, [P, P, P, F32, P]),
     "onebit_adam_compressed_step_host": (INT, [P, P, P, P, P, F32, P]),
+    "onebit_adam_host_wait": (INT, [P, P]),
     "onebit_adam_get_state": (INT, [P, I32, P, P]),
     "onebit_adam_get_chunk_state": (INT, [P, I32, I64, P, P]),
     "onebit_adam_set_state": (INT, [P, I32, P, P]),

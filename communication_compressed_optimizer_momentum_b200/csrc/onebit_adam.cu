@@ -78,6 +78,11 @@ struct onebit_adam_s {
     // per-kernel timing
     std::vector<cudaEvent_t> ev;
     int32_t tmax = 0, tcount = 0;
+    // host-buffer steps: the read-back of x runs on its own stream so that it overlaps the
+    // next step's gradient upload (created on the first host-buffer step)
+    cudaStream_t d2h = nullptr;
+    cudaEvent_t step_done = nullptr, d2h_done = nullptr;
+    bool d2h_pending = false;
 };
 
 namespace {
@@ -413,12 +418,30 @@ int onebit_adam_compressed_step_host(onebit_adam_t h, float* x_dev, void* grads_
     if (grads_host == nullptr || x_host == nullptr || grads_dev == nullptr || x_dev == nullptr)
         return ONEBIT_ERR_ARG;
     cudaStream_t st = as_stream(stream);
+    if (h->d2h == nullptr) {
+        ONEBIT_CUDA(cudaStreamCreateWithFlags(&h->d2h, cudaStreamNonBlocking));
+        ONEBIT_CUDA(cudaEventCreateWithFlags(&h->step_done, cudaEventDisableTiming));
+        ONEBIT_CUDA(cudaEventCreateWithFlags(&h->d2h_done, cudaEventDisableTiming));
+    }
     const uint64_t gbytes = (uint64_t)h->geo.W * h->geo.d * grad_elem_bytes(h->gtype);
+    // the upload is queued first, so it overlaps the previous step's read-back of x; the step
+    // itself (which rewrites x) waits for that read-back
     ONEBIT_CUDA(cudaMemcpyAsync(grads_dev, grads_host, gbytes, cudaMemcpyHostToDevice, st));
+    if (h->d2h_pending) ONEBIT_CUDA(cudaStreamWaitEvent(st, h->d2h_done, 0));
     const int rc = onebit_adam_compressed_step(h, x_dev, grads_dev, lr, stream);
     if (rc != ONEBIT_OK) return rc;
+    ONEBIT_CUDA(cudaEventRecord(h->step_done, st));
+    ONEBIT_CUDA(cudaStreamWaitEvent(h->d2h, h->step_done, 0));
     ONEBIT_CUDA(cudaMemcpyAsync(x_host, x_dev, (uint64_t)h->geo.d * sizeof(float),
-                                cudaMemcpyDeviceToHost, st));
+                                cudaMemcpyDeviceToHost, h->d2h));
+    ONEBIT_CUDA(cudaEventRecord(h->d2h_done, h->d2h));
+    h->d2h_pending = true;
+    return ONEBIT_OK;
+}
+
+int onebit_adam_host_wait(onebit_adam_t h, void* stream) {
+    if (!valid_handle(h)) return ONEBIT_ERR_ARG;
+    if (h->d2h_pending) ONEBIT_CUDA(cudaStreamWaitEvent(as_stream(stream), h->d2h_done, 0));
     return ONEBIT_OK;
 }
 
@@ -622,6 +645,12 @@ int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps) {
 void onebit_adam_destroy(onebit_adam_t h) {
     if (h == nullptr) return;
     free_events(h);
+    if (h->d2h != nullptr) {
+        cudaStreamSynchronize(h->d2h);
+        cudaStreamDestroy(h->d2h);
+        cudaEventDestroy(h->step_done);
+        cudaEventDestroy(h->d2h_done);
+    }
     delete h;
 }
 

@@ -128,12 +128,18 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
 /*
  * The same compressed step fed from host memory: copies grads_host ([W][d] of the bound type,
  * pinned host memory for an asynchronous copy) into grads_dev, runs the step on x_dev, and
- * copies the updated x_dev back into x_host (fp32[d]). All copies and kernels are queued on
- * `stream`; the host buffers must not be touched until the stream has finished.
+ * copies the updated x_dev back into x_host (fp32[d]). The upload and the step are queued on
+ * `stream`; the read-back of x runs on a stream of the handle (created on the first call), so
+ * that it overlaps the next call's upload, and the next call's step waits for it. x_host holds
+ * this step's result once onebit_adam_host_wait(h, s) has been called and `s` has finished (or
+ * the device is synchronized); grads_host may be reused once `stream` has finished.
  */
 int onebit_adam_compressed_step_host(onebit_adam_t h, float* x_dev, void* grads_dev,
                                      const void* grads_host, float* x_host, float lr,
                                      void* stream);
+
+/* Make `stream` wait for the last host-buffer step's read-back of x (no-op if there is none). */
+int onebit_adam_host_wait(onebit_adam_t h, void* stream);
 
 /*
  * Copy one piece of state into dst (device memory, contiguous, the size listed in

@@ -215,8 +215,19 @@ def test_host_entry_matches_device_entry():
         a.step(xa, g, 1e-3)
         g_host = g.cpu().pin_memory()
         b.step_host(xb, gdev, g_host, x_host, 1e-3)
-        torch.cuda.synchronize()
+        b.host_wait()
+        torch.cuda.current_stream().synchronize()
         assert torch.equal(x_host, xa.cpu())
+    assert torch.equal(xa, xb)
+    # back-to-back host steps: each read-back overlaps the next upload; the results still match
+    hosts = [g.cpu().pin_memory() for g in gl]
+    outs = [torch.empty(d, pin_memory=True) for _ in gl]
+    for g, gh, xo in zip(gl, hosts, outs):
+        a.step(xa, g, 1e-3)
+        b.step_host(xb, gdev, gh, xo, 1e-3)
+    b.host_wait()
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(outs[-1], xa.cpu())
     assert torch.equal(xa, xb)
     a.close()
     b.close()
