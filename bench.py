@@ -233,11 +233,12 @@ def run_ours(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        # one replica per GPU; NCCL carries only the barriers and the max-over-ranks timing
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
     wl = get_workload(args.workload, args.scale_d)
     dt = wls.torch_dtype(wl)
 
