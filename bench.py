@@ -206,6 +206,20 @@ def _to_np(t):
     return t.numpy().copy()
 
 
+def host_cpu():
+    """Model string and logical CPU count of the host the CPU baseline runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "nproc": os.cpu_count()}
+
+
 def oracle_sample_rate(wl, state, g, seconds):
     """Time oracle compressed steps on one chunk-sized problem until `seconds` have passed
     (at least one step). Returns (params*workers/s, steps, elements per step)."""
@@ -349,7 +363,8 @@ def run_ours(args):
         rate, n_steps, n = oracle_sample_rate(wl, st, gk, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "chunk 0 of the workload (%d params x %d workers), %d oracle "
-                         "compressed step(s), single-threaded C" % (n, wl.W, n_steps)}
+                         "compressed step(s), single-threaded C" % (n, wl.W, n_steps),
+               "host": host_cpu()}
 
     if rank == 0:
         from communication_compressed_optimizer_momentum_b200 import workloads as _w
@@ -414,7 +429,8 @@ def run_reference(args):
         "config": dict(wls.describe(wl), sample_d=n, sample_C=sw.C),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                          "sample": "%d params x %d workers (one chunk) of %s per step, "
-                                   "single-threaded C oracle" % (n, sw.W, wl.name)},
+                                   "single-threaded C oracle" % (n, sw.W, wl.name),
+                         "host": host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
