@@ -168,6 +168,69 @@ def onebit_adam_destroy(h) -> None:
     _abi.lib().onebit_adam_destroy(_handle(h))
 
 
+def onebit_dp_chunk_range(nch: int, R: int, q: int) -> Tuple[int, int]:
+    k0, k1 = ctypes.c_int64(), ctypes.c_int64()
+    _check(_abi.lib().onebit_dp_chunk_range(nch, R, q, ctypes.byref(k0), ctypes.byref(k1)),
+           "onebit_dp_chunk_range")
+    return k0.value, k1.value
+
+
+def onebit_dp_init(d: int, W: int, C: int, beta1: float, beta2: float, eps: float, R: int,
+                   rank: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_abi.lib().onebit_dp_init(ctypes.byref(h), d, W, C, beta1, beta2, eps, R, rank),
+           "onebit_dp_init")
+    return h
+
+
+def onebit_dp_info(h) -> dict:
+    out = (ctypes.c_int64 * 8)()
+    _check(_abi.lib().onebit_dp_info(_handle(h), out), "onebit_dp_info")
+    keys = ("R", "rank", "W", "k0", "k1", "e0", "d_own", "exchange_bytes")
+    return dict(zip(keys, list(out)))
+
+
+def onebit_dp_exchange(h) -> Tuple[int, int]:
+    base, n = ctypes.c_void_p(), ctypes.c_uint64()
+    _check(_abi.lib().onebit_dp_exchange(_handle(h), ctypes.byref(base), ctypes.byref(n)),
+           "onebit_dp_exchange")
+    return base.value, n.value
+
+
+def onebit_dp_ipc_handle(h) -> bytes:
+    buf = ctypes.create_string_buffer(64)
+    _check(_abi.lib().onebit_dp_ipc_handle(_handle(h), buf), "onebit_dp_ipc_handle")
+    return buf.raw
+
+
+def onebit_dp_open_peer(h, q: int, handle: bytes) -> None:
+    buf = ctypes.create_string_buffer(bytes(handle), 64)
+    _check(_abi.lib().onebit_dp_open_peer(_handle(h), q, buf), "onebit_dp_open_peer")
+
+
+def onebit_dp_set_peer(h, q: int, base: int) -> None:
+    _check(_abi.lib().onebit_dp_set_peer(_handle(h), q, ctypes.c_void_p(base)),
+           "onebit_dp_set_peer")
+
+
+def onebit_dp_connect(h, stream=None) -> None:
+    _check(_abi.lib().onebit_dp_connect(_handle(h), _stream(stream)), "onebit_dp_connect")
+
+
+def onebit_dp_set_timeout(h, timeout_us: int) -> None:
+    _check(_abi.lib().onebit_dp_set_timeout(_handle(h), timeout_us), "onebit_dp_set_timeout")
+
+
+def onebit_dp_warmup_phase(h, phase: int, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit_dp_warmup_phase(_handle(h), phase, _ptr(x), _ptr(grads), lr,
+                                             _stream(stream)), "onebit_dp_warmup_phase")
+
+
+def onebit_dp_compressed_phase(h, phase: int, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit_dp_compressed_phase(_handle(h), phase, _ptr(x), _ptr(grads), lr,
+                                                 _stream(stream)), "onebit_dp_compressed_phase")
+
+
 def onebit_strerror(code: int) -> str:
     return _abi.lib().onebit_strerror(code).decode()
 
@@ -232,11 +295,15 @@ class OneBitAdam:
 
     def __init__(self, d: int, W: int, C: int, beta1: float = 0.9, beta2: float = 0.999,
                  eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None):
+        self._setup(onebit_adam_init(d, W, C, beta1, beta2, eps), d, W, C, grad_dtype, device,
+                    stream)
+
+    def _setup(self, h, d, W, C, grad_dtype, device, stream):
         import torch
         grad_dtype = torch.float32 if grad_dtype is None else grad_dtype
         self.d, self.W, self.C = d, W, C
         self.grad_dtype = grad_dtype
-        self.h = onebit_adam_init(d, W, C, beta1, beta2, eps)
+        self.h = h
         code = dtype_code(grad_dtype)
         nbytes = onebit_adam_workspace_bytes(self.h, code)
         raw = torch.empty(nbytes + 256, dtype=torch.uint8, device=device)

@@ -40,6 +40,17 @@ SIGNATURES = {
     "onebit_unpack": (INT, [P, P, I64, I64, P, P]),
     "onebit_compress_static": (INT, [P, I64, I64, P, P, P]),
     "onebit_selftest_bounded_wait": (INT, [I32, P, P]),
+    "onebit_dp_chunk_range": (INT, [I64, I32, I32, ctypes.POINTER(I64), ctypes.POINTER(I64)]),
+    "onebit_dp_init": (INT, [ctypes.POINTER(P), I64, I32, I64, F32, F32, F32, I32, I32]),
+    "onebit_dp_info": (INT, [P, ctypes.POINTER(I64)]),
+    "onebit_dp_exchange": (INT, [P, ctypes.POINTER(P), U64P]),
+    "onebit_dp_ipc_handle": (INT, [P, P]),
+    "onebit_dp_open_peer": (INT, [P, I32, P]),
+    "onebit_dp_set_peer": (INT, [P, I32, P]),
+    "onebit_dp_connect": (INT, [P, P]),
+    "onebit_dp_set_timeout": (INT, [P, ctypes.c_uint64]),
+    "onebit_dp_warmup_phase": (INT, [P, I32, P, P, F32, P]),
+    "onebit_dp_compressed_phase": (INT, [P, I32, P, P, F32, P]),
     "onebit_strerror": (ctypes.c_char_p, [I32]),
     "onebit_last_error": (ctypes.c_char_p, []),
 }

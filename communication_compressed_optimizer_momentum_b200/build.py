@@ -15,7 +15,8 @@ SRC_DIR = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libonebit_adam.so")
 SOURCES = [os.path.join(SRC_DIR, "onebit_adam.cu")]
-DEPS = SOURCES + [os.path.join(SRC_DIR, "kernels.cuh"), os.path.join(INCLUDE, "onebit_adam.h")]
+DEPS = SOURCES + [os.path.join(SRC_DIR, "kernels.cuh"), os.path.join(SRC_DIR, "kernels_dp.cuh"),
+                  os.path.join(INCLUDE, "onebit_adam.h")]
 
 # --fmad=false: no contraction of the method's fp32 multiply-adds (every fp32 operation is one
 # IEEE operation); fp64 fused multiply-adds are written out where wanted. No fast-math, so

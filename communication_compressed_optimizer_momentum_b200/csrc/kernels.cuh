@@ -52,6 +52,39 @@ struct Geometry {
 };
 
 // ------------------------------------------------------------------------------------------
+// Data-parallel ranks. With R ranks (one per GPU), rank q holds W / R of the workers and serves
+// the chunks [kb[q], kb[q + 1]): the compressed allreduce becomes an exchange of plane slices
+// and scales (worker side -> the chunk's server) and a broadcast of the server plane and scales
+// (server -> every rank), written by the kernels straight into the peers' memory. The route
+// lists, per rank, the addresses (in this process: mapped peer memory, or this GPU's own
+// memory when ranks are emulated on one GPU) of the buffers the peers write.
+
+constexpr int kMaxRanks = 8;
+
+struct DpRoute {
+    int32_t R, rank;          // ranks, this rank
+    int32_t w0;               // global index of this rank's first worker
+    int32_t W;                // workers over all ranks
+    int64_t kb[kMaxRanks + 1];      // chunk bounds of the ranks
+    int64_t ldw[kMaxRanks];         // receive-plane row length (words) at rank q
+    uint32_t* planes[kMaxRanks];    // rank q's receive planes [W][ldw[q]]
+    float* scales[kMaxRanks];       // rank q's receive scales [W][kb[q+1] - kb[q]]
+    uint32_t* bits_s[kMaxRanks];    // rank q's server plane over all chunks
+    float* S[kMaxRanks];            // rank q's server scales over all chunks
+    float* m[kMaxRanks];            // rank q's momentum
+    float* v[kMaxRanks];            // rank q's variance
+    const double* wpart[kMaxRanks];  // rank q's warm-up gradient sums over its workers
+    uint32_t* flags[kMaxRanks];     // rank q's barrier flags, one per sending rank
+};
+
+// The rank that serves chunk k (ranks with an empty range are skipped).
+__device__ __forceinline__ int dp_owner(const DpRoute* rt, int64_t k) {
+    int q = 0;
+    while (q + 1 < rt->R && k >= rt->kb[q + 1]) ++q;
+    return q;
+}
+
+// ------------------------------------------------------------------------------------------
 // small helpers
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -142,6 +175,7 @@ struct WorkerArgs {
     uint32_t* bits_w;     // [W][ldw]
     double* part_w;       // [W][nch][nseg]
     uint32_t* status;
+    const DpRoute* route;  // data-parallel ranks only: where the plane words go
 };
 
 // Gradient loads of N consecutive elements (N = 4 or 8), fp32 or bf16 bit patterns (uint16_t,
@@ -205,7 +239,10 @@ template <bool VEC> struct GradLoadN<uint16_t, VEC, 8> {
 // LAZY_M: the shared momentum is the decompressed server message of the previous step, m =
 // (bit ? S_k : -S_k), rebuilt here from the server plane instead of read as fp32 (4 bytes per
 // parameter fewer to read, and k_apply need not write it).
-template <typename GT, bool VEC, bool LAZY_M, int EPT>
+// DP: the worker rows are this rank's W / R workers, and the plane words of chunk k go to row
+// (w0 + w) of the receive planes of the rank that serves chunk k (a store to peer memory), so
+// that the exchange of the compressed allreduce travels with the compression itself.
+template <typename GT, bool VEC, bool LAZY_M, int EPT, bool DP = false>
 __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const WorkerArgs a) {
     constexpr int ITEMS = kSeg / (kThreads * EPT);
     constexpr int LPW = 32 / EPT;  // lanes that share one 32-element sign word
@@ -246,11 +283,22 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
     }
     const float b1 = a.beta1, omb1 = a.omb1;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
+    uint32_t* bw0;
+    int64_t bld;
+    if constexpr (DP) {
+        const DpRoute* rt = a.route;
+        const int q = dp_owner(rt, k);
+        bld = rt->ldw[q];
+        bw0 = rt->planes[q] + (int64_t)rt->w0 * bld + ((base - rt->kb[q] * a.geo.C) >> 5);
+    } else {
+        bld = a.geo.ldw;
+        bw0 = a.bits_w + (base >> 5);
+    }
     for (int w = 0; w < W; ++w) {
         const float sp = a.s_lazy[(int64_t)w * a.geo.nch + k];
         const GT* gw = g0 + (int64_t)w * a.geo.d;
         float* ew = a.ew + (int64_t)w * a.geo.ld + base;
-        uint32_t* bw = a.bits_w + (int64_t)w * a.geo.ldw + (base >> 5);
+        uint32_t* bw = bw0 + (int64_t)w * bld;
         double ss = 0.0;
 #pragma unroll
         for (int it = 0; it < ITEMS; ++it) {
@@ -297,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
         ss = warp_sum(ss);
         if (lane == 0) red_w[w * kWarps + warp] = ss;
     }
+    if constexpr (DP) __threadfence_system();  // peer stores before the rank's barrier signal
     __syncthreads();
     bool nan_seen = false;
     for (int w = tid; w < W; w += kThreads) {
@@ -312,15 +361,13 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
 // reduce one row (row = w * nch + k for the workers, k for the server). Writes the reported
 // scale and the scale that rebuilds the lazy residual next step.
 
+// The scale of row r (active rows only; every thread of the row returns it). The TPR threads of
+// the row sum its nseg-strided partials in a fixed order.
 template <int TPR>
-__global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t rows,
-                                                     int64_t nch, int64_t nseg, int64_t seg,
-                                                     int64_t C, int64_t d, float* out,
-                                                     float* lazy) {
-    __shared__ double red[kWarps];
-    const int64_t r = (int64_t)blockIdx.x * (kThreads / TPR) + threadIdx.x / TPR;
+__device__ __forceinline__ float row_scale(const double* part, int64_t r, bool active,
+                                           int64_t nch, int64_t nseg, int64_t seg, int64_t C,
+                                           int64_t d, double* red) {
     const int sub = threadIdx.x % TPR;
-    const bool active = r < rows;
     int64_t clen = 1;
     double acc = 0.0;
     if (active) {
@@ -336,11 +383,50 @@ __global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t
         __syncthreads();
         acc = block_total(red);
     }
-    if (active && sub == 0) {
-        const float s = __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)clen)));
+    return __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)clen)));
+}
+
+template <int TPR>
+__global__ void __launch_bounds__(kThreads) k_scales(const double* part, int64_t rows,
+                                                     int64_t nch, int64_t nseg, int64_t seg,
+                                                     int64_t C, int64_t d, float* out,
+                                                     float* lazy) {
+    __shared__ double red[kWarps];
+    const int64_t r = (int64_t)blockIdx.x * (kThreads / TPR) + threadIdx.x / TPR;
+    const bool active = r < rows;
+    const float s = row_scale<TPR>(part, r, active, nch, nseg, seg, C, d, red);
+    if (active && threadIdx.x % TPR == 0) {
         out[r] = s;
         lazy[r] = s;
     }
+}
+
+// Data-parallel scales. Workers (SERVER false; rows = this rank's workers x all chunks): the
+// scale is also stored in the serving rank's receive scales, row w0 + w. Server (SERVER true;
+// rows = this rank's chunks): the scale is broadcast into every rank's server scales; `out` is
+// not used (the broadcast includes this rank's own copy).
+template <int TPR, bool SERVER>
+__global__ void __launch_bounds__(kThreads) k_scales_dp(const double* part, int64_t rows,
+                                                        int64_t nch, int64_t nseg, int64_t seg,
+                                                        int64_t C, int64_t d, float* out,
+                                                        float* lazy, const DpRoute* rt) {
+    __shared__ double red[kWarps];
+    const int64_t r = (int64_t)blockIdx.x * (kThreads / TPR) + threadIdx.x / TPR;
+    const bool active = r < rows;
+    const float s = row_scale<TPR>(part, r, active, nch, nseg, seg, C, d, red);
+    if (active && threadIdx.x % TPR == 0) {
+        lazy[r] = s;
+        if constexpr (SERVER) {
+            const int64_t kg = rt->kb[rt->rank] + r;
+            for (int p = 0; p < rt->R; ++p) rt->S[p][kg] = s;
+        } else {
+            out[r] = s;
+            const int64_t w = r / nch, k = r - w * nch;
+            const int q = dp_owner(rt, k);
+            rt->scales[q][(rt->w0 + w) * (rt->kb[q + 1] - rt->kb[q]) + (k - rt->kb[q])] = s;
+        }
+    }
+    __threadfence_system();
 }
 
 // ------------------------------------------------------------------------------------------
@@ -447,6 +533,7 @@ struct ServerArgs {
     uint32_t* bits_s;        // [ldw]
     double* part_s;          // [nch][blocks per chunk]: one fp64 partial per block
     uint32_t* status;
+    const DpRoute* route;    // data-parallel ranks only: where the server plane goes
 };
 
 // Pipeline depth of k_server: two stages while they fit next to the tables and a block has
@@ -528,7 +615,10 @@ __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stag
     if (STAGE_RES) bulk_load(stage + (size_t)wpad * kTileRow, a.es + base, es_bytes, bar);
 }
 
-template <bool POW2, bool STAGE_RES>
+// BCAST (data-parallel ranks): the geometry is this rank's range of chunks, the plane rows are
+// the receive planes of all W workers, and every server plane word is stored into every rank's
+// server plane (the broadcast half of the compressed allreduce, to peer memory).
+template <bool POW2, bool STAGE_RES, bool BCAST = false>
 __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     extern __shared__ __align__(16) unsigned char smem_srv[];
     const int W = a.geo.W;
@@ -776,7 +866,15 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 uint32_t word = byte << (8 * (lane & 3));
                 word |= __shfl_xor_sync(kFull, word, 1);
                 word |= __shfl_xor_sync(kFull, word, 2);
-                if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
+                if ((lane & 3) == 0 && nv > 0) {
+                    if constexpr (BCAST) {
+                        const DpRoute* rt = a.route;
+                        const int64_t gw = ((rt->kb[rt->rank] * a.geo.C) >> 5) + wbase + wd;
+                        for (int p = 0; p < rt->R; ++p) rt->bits_s[p][gw] = word;
+                    } else {
+                        a.bits_s[wbase + wd] = word;
+                    }
+                }
             }
         }
         // everyone is done with this stage (or some thread's wait expired: then all leave,
@@ -793,6 +891,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             server_issue<STAGE_RES>(a, stages + (size_t)st * stage_words, wpad, &bars[st], c0,
                                     clen, j0 + t + nst);
     }
+    if constexpr (BCAST) __threadfence_system();  // peer stores before the barrier signal
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
@@ -872,13 +971,55 @@ struct WarmupArgs {
     float* x;       // [d] caller-owned
 };
 
-// EPT elements per thread as in k_worker (8 for bf16, 4 for fp32 gradients). The fp64 sum over
-// workers runs in worker order (bit-exact with the definition); the gradient loads of UNR
-// workers are issued together so that they are in flight at once.
+// fp64 sum over the W gradient rows (row stride d) of EPT consecutive elements at offset off,
+// nv of them valid, in worker order (bit-exact with the definition); the loads of UNR workers
+// are issued together so that they are in flight at once.
+template <typename GT, bool VEC, int EPT>
+__device__ __forceinline__ void worker_grad_sum(const GT* g0, int64_t d, int W, int64_t off,
+                                                int nv, double (&acc)[EPT]) {
+    constexpr int UNR = 4;
+#pragma unroll
+    for (int c = 0; c < EPT; ++c) acc[c] = 0.0;
+    int w = 0;
+    if constexpr (sizeof(GT) == 2 && VEC && EPT == 8) {
+        for (; w + UNR <= W && nv == EPT; w += UNR) {
+            uint4 raw[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u)
+                raw[u] = *reinterpret_cast<const uint4*>(g0 + (int64_t)(w + u) * d + off);
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const uint32_t r[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    acc[2 * h] = __dadd_rn(acc[2 * h], bf16_to_f64(r[h] & 0xffffu));
+                    acc[2 * h + 1] = __dadd_rn(acc[2 * h + 1], bf16_to_f64(r[h] >> 16));
+                }
+            }
+        }
+    }
+    for (; w + UNR <= W; w += UNR) {
+        float gf[UNR][EPT];
+#pragma unroll
+        for (int u = 0; u < UNR; ++u)
+            GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)(w + u) * d + off, nv, gf[u]);
+#pragma unroll
+        for (int u = 0; u < UNR; ++u)
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[u][c]);
+    }
+    for (; w < W; ++w) {
+        float gf[EPT];
+        GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)w * d + off, nv, gf);
+#pragma unroll
+        for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[c]);
+    }
+}
+
+// EPT elements per thread as in k_worker (8 for bf16, 4 for fp32 gradients).
 template <typename GT, bool VEC, int EPT>
 __global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
     constexpr int ITEMS = kSeg / (kThreads * EPT);
-    constexpr int UNR = 4;
     int64_t k, j, base, len;
     if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x;
@@ -892,42 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
         const int nv = r <= 0 ? 0 : (r >= EPT ? EPT : (int)r);
         if (nv == 0) continue;
         double acc[EPT];
-#pragma unroll
-        for (int c = 0; c < EPT; ++c) acc[c] = 0.0;
-        int w = 0;
-        if constexpr (sizeof(GT) == 2 && VEC && EPT == 8) {
-            for (; w + UNR <= W && nv == EPT; w += UNR) {
-                uint4 raw[UNR];
-#pragma unroll
-                for (int u = 0; u < UNR; ++u)
-                    raw[u] = *reinterpret_cast<const uint4*>(g0 + (int64_t)(w + u) * a.geo.d + off);
-#pragma unroll
-                for (int u = 0; u < UNR; ++u) {
-                    const uint32_t r[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        acc[2 * h] = __dadd_rn(acc[2 * h], bf16_to_f64(r[h] & 0xffffu));
-                        acc[2 * h + 1] = __dadd_rn(acc[2 * h + 1], bf16_to_f64(r[h] >> 16));
-                    }
-                }
-            }
-        }
-        for (; w + UNR <= W; w += UNR) {
-            float gf[UNR][EPT];
-#pragma unroll
-            for (int u = 0; u < UNR; ++u)
-                GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)(w + u) * a.geo.d + off, nv, gf[u]);
-#pragma unroll
-            for (int u = 0; u < UNR; ++u)
-#pragma unroll
-                for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[u][c]);
-        }
-        for (; w < W; ++w) {
-            float gf[EPT];
-            GradLoadN<GT, VEC, EPT>::load(g0 + (int64_t)w * a.geo.d + off, nv, gf);
-#pragma unroll
-            for (int c = 0; c < EPT; ++c) acc[c] = __dadd_rn(acc[c], (double)gf[c]);
-        }
+        worker_grad_sum<GT, VEC, EPT>(g0, a.geo.d, W, off, nv, acc);
 #pragma unroll
         for (int h = 0; h < EPT / 4; ++h) {
             const int64_t o4 = off + 4 * h;

@@ -23,6 +23,7 @@
 
 #include "onebit_adam.h"
 #include "kernels.cuh"
+#include "kernels_dp.cuh"
 
 using namespace onebit;
 
@@ -32,6 +33,7 @@ thread_local std::string g_last_error;
 
 constexpr int32_t kMaxWorkers = 256;
 constexpr int kLaunchesPerStep = 5;
+constexpr int kLaunchesPerStepDp = 7;  // plus one barrier after each half of the exchange
 constexpr int kEventsPerStep = kLaunchesPerStep + 1;
 
 enum Phase { kUnbound = 0, kWarmup = 1, kCompressed = 2 };
@@ -52,10 +54,41 @@ inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
-// Workspace regions, each 256-byte aligned.
+// Workspace regions, each 256-byte aligned. For a data-parallel rank, m, v, bits_w, bits_s and
+// S_out have no space here (m, v, the server plane and scales live in the exchange region, the
+// worker planes at their servers) and `route` holds the device copy of the rank's route.
 struct Layout {
-    uint64_t m, v, es, ew, bits_w, bits_s, s_out, s_lazy, S_out, S_lazy, part_w, part_s, status;
+    uint64_t route, m, v, es, ew, bits_w, bits_s, s_out, s_lazy, S_out, S_lazy, part_w, part_s,
+        status;
     uint64_t total;
+};
+
+// Exchange region of a data-parallel rank: the buffers that other ranks write (and, for the
+// warm-up partial sums, read). Its layout depends only on (d, W, C, R), so it is the same on
+// every rank and one base address per rank locates all of a peer's buffers.
+struct XLayout {
+    uint64_t flags, m, v, wpart, planes, rscales, bits_s, S;
+    uint64_t total;
+};
+
+// The data-parallel part of a handle (R = 0: a single-GPU handle).
+struct DpState {
+    int32_t R = 0, rank = 0;
+    int32_t Wg = 0;                    // workers over all ranks
+    int64_t kb[kMaxRanks + 1] = {};    // chunk bounds of the ranks
+    Geometry gs{};                     // this rank's chunks, all Wg workers
+    int64_t e0 = 0;                    // first element of this rank's chunks
+    XLayout xl{};
+    char* xch = nullptr;               // this rank's exchange region (cudaMalloc)
+    char* peer[kMaxRanks] = {};        // peers' exchange regions, addresses in this process
+    bool ipc[kMaxRanks] = {};          // peer mapped by CUDA IPC (closed at destroy)
+    DpRoute route{};                   // host copy of the route
+    DpRoute* route_dev = nullptr;      // device copy (in the workspace)
+    bool connected = false;
+    uint32_t epoch = 0;                // barriers signalled so far
+    int next_phase = 0;                // phase-by-phase driving: the phase expected next
+    int phase_kind = 0;                // 0 none in progress, 1 warm-up, 2 compressed
+    uint64_t timeout_ns = 10000000000ull;
 };
 
 }  // namespace
@@ -83,12 +116,15 @@ struct onebit_adam_s {
     cudaStream_t d2h = nullptr;
     cudaEvent_t step_done = nullptr, d2h_done = nullptr;
     bool d2h_pending = false;
+    DpState dp;
 };
 
 namespace {
 
 Layout make_layout(const onebit_adam_s& h) {
     const Geometry& g = h.geo;
+    const bool dp = h.dp.R > 0;
+    const Geometry& gs = dp ? h.dp.gs : g;  // the server's chunks
     Layout L{};
     uint64_t off = 0;
     auto take = [&](uint64_t bytes) {
@@ -96,25 +132,71 @@ Layout make_layout(const onebit_adam_s& h) {
         off = (uint64_t)round_up((int64_t)(off + bytes), 256);
         return at;
     };
-    const uint64_t f = sizeof(float);
-    L.m = take(g.ld * f);
-    L.v = take(g.ld * f);
-    L.es = take(g.ld * f);
+    const uint64_t f = sizeof(float), u = sizeof(uint32_t);
+    L.route = take(dp ? sizeof(DpRoute) : 0);
+    L.m = take(dp ? 0 : g.ld * f);
+    L.v = take(dp ? 0 : g.ld * f);
+    L.es = take(gs.ld * f);
     L.ew = take((uint64_t)g.W * g.ld * f);
-    L.bits_w = take((uint64_t)g.W * g.ldw * sizeof(uint32_t));
-    L.bits_s = take(g.ldw * sizeof(uint32_t));
+    L.bits_w = take(dp ? 0 : (uint64_t)g.W * g.ldw * u);
+    L.bits_s = take(dp ? 0 : g.ldw * u);
     L.s_out = take((uint64_t)g.W * g.nch * f);
     L.s_lazy = take((uint64_t)g.W * g.nch * f);
-    L.S_out = take(g.nch * f);
-    L.S_lazy = take(g.nch * f);
+    L.S_out = take(dp ? 0 : g.nch * f);
+    L.S_lazy = take((uint64_t)std::max<int64_t>(gs.nch, 1) * f);
     L.part_w = take((uint64_t)g.W * g.nch * g.nseg * sizeof(double));
-    L.part_s = take((uint64_t)g.nch * g.nseg_s * sizeof(double));
+    L.part_s = take((uint64_t)std::max<int64_t>(gs.nch, 1) * g.nseg_s * sizeof(double));
     L.status = take(4 * sizeof(uint32_t));
     L.total = off;
     return L;
 }
 
+// Rank q's chunks of nch: [q * nch / R, (q + 1) * nch / R), contiguous and balanced.
+void dp_range(int64_t nch, int32_t R, int32_t q, int64_t* k0, int64_t* k1) {
+    *k0 = (int64_t)((__int128)nch * q / R);
+    *k1 = (int64_t)((__int128)nch * (q + 1) / R);
+}
+
+// Elements and receive-plane row length (words, padded to 16 bytes) of rank q's chunks.
+int64_t dp_elems(const onebit_adam_s& h, int32_t q) {
+    const Geometry& g = h.geo;
+    const int64_t* kb = h.dp.kb;
+    return std::max<int64_t>(0, std::min(kb[q + 1] * g.C, g.d) - kb[q] * g.C);
+}
+int64_t dp_ldw(const onebit_adam_s& h, int32_t q) {
+    return round_up(std::max<int64_t>(ceil_div(dp_elems(h, q), 32), 1), 4);
+}
+
+XLayout make_xlayout(const onebit_adam_s& h) {
+    const Geometry& g = h.geo;
+    const DpState& dp = h.dp;
+    int64_t ldw_max = 4, nch_max = 1;
+    for (int32_t q = 0; q < dp.R; ++q) {
+        ldw_max = std::max(ldw_max, dp_ldw(h, q));
+        nch_max = std::max(nch_max, dp.kb[q + 1] - dp.kb[q]);
+    }
+    XLayout X{};
+    uint64_t off = 0;
+    auto take = [&](uint64_t bytes) {
+        const uint64_t at = off;
+        off = (uint64_t)round_up((int64_t)(off + bytes), 256);
+        return at;
+    };
+    const uint64_t f = sizeof(float), u = sizeof(uint32_t);
+    X.flags = take(kMaxRanks * u);
+    X.m = take(g.ld * f);
+    X.v = take(g.ld * f);
+    X.wpart = take(g.ld * sizeof(double));
+    X.planes = take((uint64_t)dp.Wg * ldw_max * u);
+    X.rscales = take((uint64_t)dp.Wg * nch_max * f);
+    X.bits_s = take(g.ldw * u);
+    X.S = take(g.nch * f);
+    X.total = off;
+    return X;
+}
+
 bool valid_handle(onebit_adam_t h) { return h != nullptr; }
+bool is_dp(const onebit_adam_s* h) { return h->dp.R > 0; }
 
 int64_t step_blocks(const Geometry& g) { return g.nch * g.nseg; }
 int64_t server_blocks_per_chunk(const Geometry& g) {
@@ -129,6 +211,13 @@ ServerKernel server_kernel(int W) {
     const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W);
     if (pow2) return staged ? k_server<true, true> : k_server<true, false>;
     return staged ? k_server<false, true> : k_server<false, false>;
+}
+
+// The same for a data-parallel rank: the server plane is broadcast to every rank.
+ServerKernel server_kernel_dp(int W) {
+    const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W);
+    if (pow2) return staged ? k_server<true, true, true> : k_server<true, false, true>;
+    return staged ? k_server<false, true, true> : k_server<false, false, true>;
 }
 
 // Launch the chunk-scale reduction (nseg partials of seg elements per row) with the thread
@@ -150,35 +239,62 @@ int launch_scales(const Geometry& g, const double* part, int64_t rows, int64_t n
     return ONEBIT_OK;
 }
 
+// Data-parallel scales (see k_scales_dp): geometry (nch, C, d) of the rows' chunks.
+template <bool SERVER>
+int launch_scales_dp(int64_t nch, int64_t C, int64_t d, const double* part, int64_t rows,
+                     int64_t nseg, int64_t seg, float* out, float* lazy, const DpRoute* rt,
+                     cudaStream_t st) {
+    if (rows == 0) return ONEBIT_OK;
+    if (nseg <= 8) {
+        k_scales_dp<1, SERVER><<<(unsigned)ceil_div(rows, kThreads), kThreads, 0, st>>>(
+            part, rows, nch, nseg, seg, C, d, out, lazy, rt);
+    } else if (nseg <= 1024) {
+        k_scales_dp<32, SERVER><<<(unsigned)ceil_div(rows, kWarps), kThreads, 0, st>>>(
+            part, rows, nch, nseg, seg, C, d, out, lazy, rt);
+    } else {
+        k_scales_dp<kThreads, SERVER><<<(unsigned)rows, kThreads, 0, st>>>(
+            part, rows, nch, nseg, seg, C, d, out, lazy, rt);
+    }
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
 // Vector width of the worker kernel: 8 elements per thread (16-byte loads of 8 bf16 values)
 // when bf16 gradient rows are 16-byte aligned, 4 (16-byte loads of 4 fp32 values, or 8-byte
 // loads of 4 bf16 values) when rows are 16- or 8-byte aligned, element by element otherwise.
-template <typename GT, bool LAZY_M>
+template <typename GT, bool LAZY_M, bool DP>
 void launch_worker_t(onebit_adam_s* h, const WorkerArgs& a, unsigned blocks, size_t smem,
                      cudaStream_t st) {
     const int64_t d = h->geo.d;
     if constexpr (sizeof(GT) == 2) {
         if (d % 8 == 0) {
-            k_worker<GT, true, LAZY_M, 8><<<blocks, kThreads, smem, st>>>(a);
+            k_worker<GT, true, LAZY_M, 8, DP><<<blocks, kThreads, smem, st>>>(a);
             return;
         }
     }
     if (d % kVec == 0)
-        k_worker<GT, true, LAZY_M, 4><<<blocks, kThreads, smem, st>>>(a);
+        k_worker<GT, true, LAZY_M, 4, DP><<<blocks, kThreads, smem, st>>>(a);
     else
-        k_worker<GT, false, LAZY_M, 4><<<blocks, kThreads, smem, st>>>(a);
+        k_worker<GT, false, LAZY_M, 4, DP><<<blocks, kThreads, smem, st>>>(a);
 }
 
 template <typename GT>
 int launch_worker(onebit_adam_s* h, const void* grads, cudaStream_t st) {
     WorkerArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->m, h->bits_s, h->S_out, grads, h->ew,
-                 h->s_lazy, h->bits_w, h->part_w, h->status};
+                 h->s_lazy, h->bits_w, h->part_w, h->status, h->dp.route_dev};
     const size_t smem = (size_t)h->geo.W * kWarps * sizeof(double);
     const unsigned blocks = (unsigned)step_blocks(h->geo);
-    if (h->m_explicit)
-        launch_worker_t<GT, false>(h, a, blocks, smem, st);
-    else
-        launch_worker_t<GT, true>(h, a, blocks, smem, st);
+    if (is_dp(h)) {
+        if (h->m_explicit)
+            launch_worker_t<GT, false, true>(h, a, blocks, smem, st);
+        else
+            launch_worker_t<GT, true, true>(h, a, blocks, smem, st);
+    } else {
+        if (h->m_explicit)
+            launch_worker_t<GT, false, false>(h, a, blocks, smem, st);
+        else
+            launch_worker_t<GT, true, false>(h, a, blocks, smem, st);
+    }
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }
@@ -228,9 +344,11 @@ uint64_t grad_elem_bytes(int32_t gtype) { return gtype == ONEBIT_BF16 ? 2 : 4; }
 
 // Explicit residuals of elements [i0, i0 + n) of every row (W rows for the workers, 1 for the
 // server) into dst[rows][n].
+// For a data-parallel rank the server residual covers the rank's own chunks only, and i0 counts
+// from their first element.
 int launch_materialize(onebit_adam_s* h, bool workers, int64_t i0, int64_t n, float* dst,
                        cudaStream_t st) {
-    const Geometry& g = h->geo;
+    const Geometry& g = workers || !is_dp(h) ? h->geo : h->dp.gs;
     const int64_t rows = workers ? g.W : 1;
     const int64_t total = rows * n;
     if (total == 0) return ONEBIT_OK;
@@ -239,6 +357,128 @@ int launch_materialize(onebit_adam_s* h, bool workers, int64_t i0, int64_t n, fl
                                                workers ? h->s_lazy : h->S_lazy, g.nch, g.C, i0,
                                                n, rows, dst);
     ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+// Worker planes of a data-parallel rank, rebuilt from the stored x_w (bit = x_w >= 0): rows of
+// elements [i0, i0 + n) into dst[W][ceil(n / 32)].
+int launch_pack_rows(onebit_adam_s* h, int64_t i0, int64_t n, uint32_t* dst, cudaStream_t st) {
+    const Geometry& g = h->geo;
+    if (n == 0) return ONEBIT_OK;
+    const int64_t nwk = ceil_div(n, 32);
+    for (int32_t w = 0; w < g.W; ++w)
+        k_pack<<<(unsigned)ceil_div(n, kSeg), kThreads, 0, st>>>(h->ew + (int64_t)w * g.ld + i0,
+                                                                 n, dst + (int64_t)w * nwk);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+// ------------------------------------------------------------------------------------------
+// Data-parallel step sequences. Phase p of a step runs on this rank alone up to the point
+// where it needs the other ranks' stores; `sig` ends the phase with this rank's barrier signal
+// and `wait` starts it with the wait for every rank's signal. A whole step fuses each signal
+// with the following wait into one barrier launch.
+
+int dp_barrier(onebit_adam_s* h, int mode, cudaStream_t st) {
+    DpState& dp = h->dp;
+    if (mode & kBarrierSignal) ++dp.epoch;
+    k_dp_barrier<<<1, 32, 0, st>>>(dp.route_dev, dp.epoch, mode, dp.timeout_ns, h->status);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+template <typename GT>
+int dp_warmup_partial(onebit_adam_s* h, const void* grads, cudaStream_t st) {
+    const Geometry& g = h->geo;
+    double* wpart = reinterpret_cast<double*>(h->dp.xch + h->dp.xl.wpart);
+    const unsigned blocks = (unsigned)step_blocks(g);
+    if constexpr (sizeof(GT) == 2) {
+        if (g.d % 8 == 0) {
+            k_warmup_partial<GT, true, 8><<<blocks, kThreads, 0, st>>>(g, grads, wpart);
+            ONEBIT_CUDA(cudaGetLastError());
+            return ONEBIT_OK;
+        }
+    }
+    if (g.d % kVec == 0)
+        k_warmup_partial<GT, true, 4><<<blocks, kThreads, 0, st>>>(g, grads, wpart);
+    else
+        k_warmup_partial<GT, false, 4><<<blocks, kThreads, 0, st>>>(g, grads, wpart);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+int dp_warmup_phase(onebit_adam_s* h, int phase, float* x, const void* grads, float lr,
+                    int mode_in, int mode_out, cudaStream_t st) {
+    DpState& dp = h->dp;
+    int rc = ONEBIT_OK;
+    if (mode_in) rc = dp_barrier(h, mode_in, st);
+    if (rc != ONEBIT_OK) return rc;
+    if (phase == 0) {
+        rc = h->gtype == ONEBIT_BF16 ? dp_warmup_partial<uint16_t>(h, grads, st)
+                                     : dp_warmup_partial<float>(h, grads, st);
+    } else if (phase == 1) {
+        if (dp.gs.d > 0) {
+            WarmupDpArgs a{dp.gs, dp.e0, h->beta1, 1.0f - h->beta1, h->beta2, 1.0f - h->beta2,
+                           dp.route_dev};
+            k_warmup_reduce<<<(unsigned)step_blocks(dp.gs), kThreads, 0, st>>>(a);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+    } else {
+        WarmupApplyArgs a{h->geo, h->eps, lr, h->m, h->v, x};
+        k_warmup_apply<<<(unsigned)step_blocks(h->geo), kThreads, 0, st>>>(a);
+        ONEBIT_CUDA(cudaGetLastError());
+    }
+    if (rc != ONEBIT_OK) return rc;
+    if (mode_out) rc = dp_barrier(h, mode_out, st);
+    return rc;
+}
+
+int dp_compressed_phase(onebit_adam_s* h, int phase, float* x, const void* grads, float lr,
+                        int mode_in, int mode_out, cudaStream_t st) {
+    DpState& dp = h->dp;
+    const Geometry& g = h->geo;
+    int rc = ONEBIT_OK;
+    if (mode_in) rc = dp_barrier(h, mode_in, st);
+    if (rc != ONEBIT_OK) return rc;
+    if (phase == 0) {
+        record(h, 0, st);
+        rc = h->gtype == ONEBIT_BF16 ? launch_worker<uint16_t>(h, grads, st)
+                                     : launch_worker<float>(h, grads, st);
+        if (rc != ONEBIT_OK) return rc;
+        record(h, 1, st);
+        rc = launch_scales_dp<false>(g.nch, g.C, g.d, h->part_w, (int64_t)g.W * g.nch, g.nseg,
+                                     kSeg, h->s_out, h->s_lazy, dp.route_dev, st);
+    } else if (phase == 1) {
+        record(h, 2, st);
+        const Geometry& gs = dp.gs;
+        if (gs.d > 0) {
+            uint32_t* planes = reinterpret_cast<uint32_t*>(dp.xch + dp.xl.planes);
+            const float* rs = reinterpret_cast<const float*>(dp.xch + dp.xl.rscales);
+            ServerArgs sa{gs, planes, rs, h->es, h->S_lazy, nullptr, h->part_s, h->status,
+                          dp.route_dev};
+            const size_t ssm = server_smem_bytes(gs.W, server_stages(gs.W, gs.nseg_s));
+            server_kernel_dp(gs.W)<<<(unsigned)server_blocks(gs), kThreads, ssm, st>>>(sa);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+        record(h, 3, st);
+        rc = launch_scales_dp<true>(gs.nch, gs.C, gs.d, h->part_s, gs.nch,
+                                    server_blocks_per_chunk(gs), kSegS * kSrvSegsPerBlock,
+                                    nullptr, h->S_lazy, dp.route_dev, st);
+    } else {
+        record(h, 4, st);
+        ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, x};
+        k_apply<<<(unsigned)step_blocks(g), kThreads, 0, st>>>(pa);
+        ONEBIT_CUDA(cudaGetLastError());
+        record(h, 5, st);
+    }
+    if (rc != ONEBIT_OK) return rc;
+    if (mode_out) rc = dp_barrier(h, mode_out, st);
+    return rc;
+}
+
+// Checks shared by the step and phase entry points of a data-parallel rank.
+int dp_ready(onebit_adam_s* h) {
+    if (!h->dp.connected) return ONEBIT_ERR_PHASE;
     return ONEBIT_OK;
 }
 
@@ -325,10 +565,35 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->part_s = reinterpret_cast<double*>(b + L.part_s);
     h->status = reinterpret_cast<uint32_t*>(b + L.status);
     h->gtype = grad_dtype;
-    const int ssm = (int)server_smem_bytes(h->geo.W, server_stages(h->geo.W, h->geo.nseg_s));
-    ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel(h->geo.W),
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     cudaStream_t st = as_stream(stream);
+    if (is_dp(h)) {
+        DpState& dp = h->dp;
+        if (dp.xch == nullptr) {
+            // the exchange region is an allocation of its own so that CUDA IPC can map it
+            void* p = nullptr;
+            ONEBIT_CUDA(cudaMalloc(&p, dp.xl.total));
+            dp.xch = static_cast<char*>(p);
+        }
+        char* x = dp.xch;
+        h->m = reinterpret_cast<float*>(x + dp.xl.m);
+        h->v = reinterpret_cast<float*>(x + dp.xl.v);
+        h->bits_s = reinterpret_cast<uint32_t*>(x + dp.xl.bits_s);
+        h->S_out = reinterpret_cast<float*>(x + dp.xl.S);
+        h->bits_w = nullptr;
+        dp.route_dev = reinterpret_cast<DpRoute*>(b + L.route);
+        dp.connected = false;
+        dp.epoch = 0;
+        dp.next_phase = 0;
+        dp.phase_kind = 0;
+        const int ssm = (int)server_smem_bytes(dp.Wg, server_stages(dp.Wg, dp.gs.nseg_s));
+        ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel_dp(dp.Wg),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
+        ONEBIT_CUDA(cudaMemsetAsync(dp.xch, 0, dp.xl.total, st));
+    } else {
+        const int ssm = (int)server_smem_bytes(h->geo.W, server_stages(h->geo.W, h->geo.nseg_s));
+        ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel(h->geo.W),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
+    }
     // m and v start at zero (Adam); the rest is cleared too so padding is deterministic.
     ONEBIT_CUDA(cudaMemsetAsync(b, 0, L.total, st));
     h->phase = kWarmup;
@@ -345,6 +610,14 @@ int onebit_adam_warmup_step(onebit_adam_t h, float* x, const void* grads, float 
     if (x == nullptr || grads == nullptr) return ONEBIT_ERR_ARG;
     if (!aligned16(x) || !aligned16(grads)) return ONEBIT_ERR_ALIGN;
     cudaStream_t st = as_stream(stream);
+    if (is_dp(h)) {
+        if (dp_ready(h) != ONEBIT_OK || h->dp.phase_kind != 0) return ONEBIT_ERR_PHASE;
+        const int both = kBarrierSignal | kBarrierWait;
+        int rc = dp_warmup_phase(h, 0, x, grads, lr, 0, both, st);
+        if (rc == ONEBIT_OK) rc = dp_warmup_phase(h, 1, x, grads, lr, 0, both, st);
+        if (rc == ONEBIT_OK) rc = dp_warmup_phase(h, 2, x, grads, lr, 0, 0, st);
+        return rc;
+    }
     return h->gtype == ONEBIT_BF16 ? launch_warmup<uint16_t>(h, x, grads, lr, st)
                                    : launch_warmup<float>(h, x, grads, lr, st);
 }
@@ -354,8 +627,16 @@ int onebit_adam_freeze_variance(onebit_adam_t h, void* stream) {
     if (h->phase != kWarmup) return ONEBIT_ERR_PHASE;
     cudaStream_t st = as_stream(stream);
     const Layout& L = h->lay;
+    if (is_dp(h) && h->dp.phase_kind != 0) return ONEBIT_ERR_PHASE;
     // residuals (lazy form: stored 0 with scale 0 rebuilds e = 0), planes, scales, partials
     ONEBIT_CUDA(cudaMemsetAsync(h->ws + L.es, 0, L.total - L.es, st));
+    if (is_dp(h)) {
+        // this rank's copy of the server plane and scales; not the receive planes and scales,
+        // which the other ranks may already be filling for the first compressed step (every
+        // word the server reads is written by its worker rank before the barrier)
+        const XLayout& X = h->dp.xl;
+        ONEBIT_CUDA(cudaMemsetAsync(h->dp.xch + X.bits_s, 0, X.total - X.bits_s, st));
+    }
     h->phase = kCompressed;
     h->steps = 0;
     return ONEBIT_OK;
@@ -380,6 +661,18 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
         Range() { nvtxRangePushA("onebit_adam_compressed_step"); }
         ~Range() { nvtxRangePop(); }
     } range;
+    if (is_dp(h)) {
+        if (dp_ready(h) != ONEBIT_OK || h->dp.phase_kind != 0) return ONEBIT_ERR_PHASE;
+        const int both = kBarrierSignal | kBarrierWait;
+        rc = dp_compressed_phase(h, 0, x, grads, lr, 0, both, st);
+        if (rc == ONEBIT_OK) rc = dp_compressed_phase(h, 1, x, grads, lr, 0, both, st);
+        if (rc == ONEBIT_OK) rc = dp_compressed_phase(h, 2, x, grads, lr, 0, 0, st);
+        if (rc != ONEBIT_OK) return rc;
+        if (h->tcount < h->tmax) ++h->tcount;
+        ++h->steps;
+        h->m_explicit = false;
+        return ONEBIT_OK;
+    }
 
     record(h, 0, st);
     rc = h->gtype == ONEBIT_BF16 ? launch_worker<uint16_t>(h, grads, st)
@@ -451,8 +744,8 @@ int onebit_adam_state_bytes(onebit_adam_t h, int32_t which, uint64_t* bytes) {
     const uint64_t f = sizeof(float);
     switch (which) {
         case ONEBIT_STATE_M:
-        case ONEBIT_STATE_V:
-        case ONEBIT_STATE_ES: *bytes = g.d * f; break;
+        case ONEBIT_STATE_V: *bytes = g.d * f; break;
+        case ONEBIT_STATE_ES: *bytes = (is_dp(h) ? h->dp.gs.d : g.d) * f; break;
         case ONEBIT_STATE_EW: *bytes = (uint64_t)g.W * g.d * f; break;
         case ONEBIT_STATE_SW: *bytes = (uint64_t)g.W * g.nch * f; break;
         case ONEBIT_STATE_SS: *bytes = g.nch * f; break;
@@ -482,6 +775,7 @@ int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* strea
         case ONEBIT_STATE_SW: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->s_out, bytes, D2D, st)); break;
         case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out, bytes, D2D, st)); break;
         case ONEBIT_STATE_BITSW:
+            if (is_dp(h)) return launch_pack_rows(h, 0, g.d, static_cast<uint32_t*>(dst), st);
             ONEBIT_CUDA(cudaMemcpy2DAsync(dst, h->nw * sizeof(uint32_t), h->bits_w,
                                           g.ldw * sizeof(uint32_t), h->nw * sizeof(uint32_t),
                                           g.W, D2D, st));
@@ -490,7 +784,8 @@ int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* strea
         case ONEBIT_STATE_EW:
         case ONEBIT_STATE_ES: {
             const bool wk = which == ONEBIT_STATE_EW;
-            const int rc2 = launch_materialize(h, wk, 0, g.d, static_cast<float*>(dst), st);
+            const int64_t n = wk || !is_dp(h) ? g.d : h->dp.gs.d;
+            const int rc2 = launch_materialize(h, wk, 0, n, static_cast<float*>(dst), st);
             if (rc2 != ONEBIT_OK) return rc2;
             break;
         }
@@ -517,14 +812,22 @@ int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void*
             break;
         case ONEBIT_STATE_V: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->v + i0, n * f, D2D, st)); break;
         case ONEBIT_STATE_EW:
+            return launch_materialize(h, true, i0, n, static_cast<float*>(dst), st);
         case ONEBIT_STATE_ES:
-            return launch_materialize(h, which == ONEBIT_STATE_EW, i0, n,
-                                      static_cast<float*>(dst), st);
+            if (is_dp(h)) {
+                // the server residual of a data-parallel rank covers its own chunks only
+                const int64_t k0 = h->dp.kb[h->dp.rank], k1 = h->dp.kb[h->dp.rank + 1];
+                if (k < k0 || k >= k1) return ONEBIT_ERR_ARG;
+                return launch_materialize(h, false, (k - k0) * g.C, n, static_cast<float*>(dst),
+                                          st);
+            }
+            return launch_materialize(h, false, i0, n, static_cast<float*>(dst), st);
         case ONEBIT_STATE_SW:
             ONEBIT_CUDA(cudaMemcpy2DAsync(dst, f, h->s_out + k, g.nch * f, f, g.W, D2D, st));
             break;
         case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out + k, f, D2D, st)); break;
         case ONEBIT_STATE_BITSW:
+            if (is_dp(h)) return launch_pack_rows(h, i0, n, static_cast<uint32_t*>(dst), st);
             ONEBIT_CUDA(cudaMemcpy2DAsync(dst, nwk * u, h->bits_w + w0, g.ldw * u, nwk * u, g.W,
                                           D2D, st));
             break;
@@ -570,7 +873,7 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
                 h->m_explicit = true;
             }
             ONEBIT_CUDA(cudaMemcpyAsync(h->es, src, bytes, D2D, st));
-            ONEBIT_CUDA(cudaMemsetAsync(h->S_lazy, 0, g.nch * f, st));
+            ONEBIT_CUDA(cudaMemsetAsync(h->S_lazy, 0, (is_dp(h) ? h->dp.gs.nch : g.nch) * f, st));
             ONEBIT_CUDA(cudaMemsetAsync(h->S_out, 0, g.nch * f, st));
             break;
         default: return ONEBIT_ERR_ARG;
@@ -600,7 +903,7 @@ int onebit_adam_info(onebit_adam_t h, int64_t out[8]) {
     out[4] = h->phase;
     out[5] = h->steps;
     out[6] = h->gtype;
-    out[7] = kLaunchesPerStep;
+    out[7] = is_dp(h) ? kLaunchesPerStepDp : kLaunchesPerStep;
     return ONEBIT_OK;
 }
 
@@ -645,6 +948,9 @@ int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps) {
 void onebit_adam_destroy(onebit_adam_t h) {
     if (h == nullptr) return;
     free_events(h);
+    for (int q = 0; q < kMaxRanks; ++q)
+        if (h->dp.ipc[q]) cudaIpcCloseMemHandle(h->dp.peer[q]);
+    if (h->dp.xch != nullptr) cudaFree(h->dp.xch);
     if (h->d2h != nullptr) {
         cudaStreamSynchronize(h->d2h);
         cudaStreamDestroy(h->d2h);
@@ -652,6 +958,209 @@ void onebit_adam_destroy(onebit_adam_t h) {
         cudaEventDestroy(h->d2h_done);
     }
     delete h;
+}
+
+// ------------------------------------------------------------------------------------------
+// Data-parallel ranks
+
+int onebit_dp_chunk_range(int64_t nch, int32_t R, int32_t q, int64_t* k0, int64_t* k1) {
+    if (nch < 0 || R < 1 || R > kMaxRanks || q < 0 || q >= R || k0 == nullptr || k1 == nullptr)
+        return ONEBIT_ERR_ARG;
+    dp_range(nch, R, q, k0, k1);
+    return ONEBIT_OK;
+}
+
+int onebit_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                   float beta2, float eps, int32_t R, int32_t rank) {
+    if (out == nullptr) return ONEBIT_ERR_ARG;
+    *out = nullptr;
+    if (R < 1 || R > kMaxRanks || rank < 0 || rank >= R) return ONEBIT_ERR_ARG;
+    if (W < 1 || W > kMaxWorkers || W % R != 0) return ONEBIT_ERR_ARG;
+    const int rc = onebit_adam_init(out, d, W / R, C, beta1, beta2, eps);
+    if (rc != ONEBIT_OK) return rc;
+    onebit_adam_s* h = *out;
+    const Geometry& g = h->geo;
+    DpState& dp = h->dp;
+    dp.R = R;
+    dp.rank = rank;
+    dp.Wg = W;
+    for (int32_t q = 0; q < R; ++q) dp_range(g.nch, R, q, &dp.kb[q], &dp.kb[q + 1]);
+    Geometry& gs = dp.gs;
+    gs.d = dp_elems(*h, rank);
+    gs.C = g.C;
+    gs.nch = dp.kb[rank + 1] - dp.kb[rank];
+    gs.nseg = g.nseg;      // the global segment counts: block partials and their reduction
+    gs.nseg_s = g.nseg_s;  // order are those of the single-GPU step
+    gs.ld = round_up(std::max<int64_t>(gs.d, 1), 64);
+    gs.ldw = dp_ldw(*h, rank);
+    gs.W = W;
+    dp.e0 = dp.kb[rank] * g.C;
+    dp.xl = make_xlayout(*h);
+    return ONEBIT_OK;
+}
+
+int onebit_dp_info(onebit_adam_t h, int64_t out[8]) {
+    if (!valid_handle(h) || out == nullptr || !is_dp(h)) return ONEBIT_ERR_ARG;
+    const DpState& dp = h->dp;
+    out[0] = dp.R;
+    out[1] = dp.rank;
+    out[2] = dp.Wg;
+    out[3] = dp.kb[dp.rank];
+    out[4] = dp.kb[dp.rank + 1];
+    out[5] = dp.e0;
+    out[6] = dp.gs.d;
+    out[7] = (int64_t)dp.xl.total;
+    return ONEBIT_OK;
+}
+
+int onebit_dp_exchange(onebit_adam_t h, void** base, uint64_t* bytes) {
+    if (!valid_handle(h) || base == nullptr || bytes == nullptr || !is_dp(h)) return ONEBIT_ERR_ARG;
+    if (h->dp.xch == nullptr) return ONEBIT_ERR_PHASE;
+    *base = h->dp.xch;
+    *bytes = h->dp.xl.total;
+    return ONEBIT_OK;
+}
+
+int onebit_dp_ipc_handle(onebit_adam_t h, void* out) {
+    if (!valid_handle(h) || out == nullptr || !is_dp(h)) return ONEBIT_ERR_ARG;
+    if (h->dp.xch == nullptr) return ONEBIT_ERR_PHASE;
+    static_assert(sizeof(cudaIpcMemHandle_t) == ONEBIT_IPC_HANDLE_BYTES, "IPC handle size");
+    cudaIpcMemHandle_t hd;
+    ONEBIT_CUDA(cudaIpcGetMemHandle(&hd, h->dp.xch));
+    std::memcpy(out, &hd, sizeof hd);
+    return ONEBIT_OK;
+}
+
+int onebit_dp_open_peer(onebit_adam_t h, int32_t q, const void* handle) {
+    if (!valid_handle(h) || handle == nullptr || !is_dp(h)) return ONEBIT_ERR_ARG;
+    DpState& dp = h->dp;
+    if (q < 0 || q >= dp.R || q == dp.rank) return ONEBIT_ERR_ARG;
+    cudaIpcMemHandle_t hd;
+    std::memcpy(&hd, handle, sizeof hd);
+    void* p = nullptr;
+    ONEBIT_CUDA(cudaIpcOpenMemHandle(&p, hd, cudaIpcMemLazyEnablePeerAccess));
+    if (dp.ipc[q]) cudaIpcCloseMemHandle(dp.peer[q]);
+    dp.peer[q] = static_cast<char*>(p);
+    dp.ipc[q] = true;
+    dp.connected = false;
+    return ONEBIT_OK;
+}
+
+int onebit_dp_set_peer(onebit_adam_t h, int32_t q, void* base) {
+    if (!valid_handle(h) || base == nullptr || !is_dp(h)) return ONEBIT_ERR_ARG;
+    DpState& dp = h->dp;
+    if (q < 0 || q >= dp.R || q == dp.rank) return ONEBIT_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(base) & 255u) != 0) return ONEBIT_ERR_ALIGN;
+    if (dp.ipc[q]) cudaIpcCloseMemHandle(dp.peer[q]);
+    dp.peer[q] = static_cast<char*>(base);
+    dp.ipc[q] = false;
+    dp.connected = false;
+    return ONEBIT_OK;
+}
+
+int onebit_dp_connect(onebit_adam_t h, void* stream) {
+    if (!valid_handle(h) || !is_dp(h)) return ONEBIT_ERR_ARG;
+    DpState& dp = h->dp;
+    if (h->phase == kUnbound || dp.xch == nullptr) return ONEBIT_ERR_PHASE;
+    for (int32_t q = 0; q < dp.R; ++q)
+        if (q != dp.rank && dp.peer[q] == nullptr) return ONEBIT_ERR_PHASE;
+    DpRoute& r = dp.route;
+    r = DpRoute{};
+    r.R = dp.R;
+    r.rank = dp.rank;
+    r.w0 = dp.rank * h->geo.W;
+    r.W = dp.Wg;
+    const XLayout& X = dp.xl;
+    for (int32_t q = 0; q <= dp.R; ++q) r.kb[q] = dp.kb[q];
+    for (int32_t q = 0; q < dp.R; ++q) {
+        char* b = q == dp.rank ? dp.xch : dp.peer[q];
+        r.ldw[q] = dp_ldw(*h, q);
+        r.planes[q] = reinterpret_cast<uint32_t*>(b + X.planes);
+        r.scales[q] = reinterpret_cast<float*>(b + X.rscales);
+        r.bits_s[q] = reinterpret_cast<uint32_t*>(b + X.bits_s);
+        r.S[q] = reinterpret_cast<float*>(b + X.S);
+        r.m[q] = reinterpret_cast<float*>(b + X.m);
+        r.v[q] = reinterpret_cast<float*>(b + X.v);
+        r.wpart[q] = reinterpret_cast<const double*>(b + X.wpart);
+        r.flags[q] = reinterpret_cast<uint32_t*>(b + X.flags);
+    }
+    ONEBIT_CUDA(cudaMemcpyAsync(dp.route_dev, &r, sizeof r, cudaMemcpyHostToDevice,
+                                as_stream(stream)));
+    dp.connected = true;
+    return ONEBIT_OK;
+}
+
+int onebit_dp_set_timeout(onebit_adam_t h, uint64_t timeout_us) {
+    if (!valid_handle(h) || !is_dp(h)) return ONEBIT_ERR_ARG;
+    if (timeout_us < 1 || timeout_us > 3600ull * 1000000ull) return ONEBIT_ERR_ARG;
+    h->dp.timeout_ns = timeout_us * 1000ull;
+    return ONEBIT_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Argument and order checks of one phase; kind 1 warm-up, 2 compressed.
+int dp_phase_check(onebit_adam_t h, int kind, int32_t phase, const float* x, const void* grads,
+                   float lr) {
+    if (!valid_handle(h) || !is_dp(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
+    if (phase < 0 || phase > 2) return ONEBIT_ERR_ARG;
+    if (h->phase != (kind == 1 ? kWarmup : kCompressed)) return ONEBIT_ERR_PHASE;
+    const DpState& dp = h->dp;
+    if (!dp.connected || phase != dp.next_phase) return ONEBIT_ERR_PHASE;
+    if (phase > 0 && dp.phase_kind != kind) return ONEBIT_ERR_PHASE;
+    if (h->geo.d == 0) return ONEBIT_OK;
+    if (phase == 0) {
+        if (grads == nullptr) return ONEBIT_ERR_ARG;
+        if (!aligned16(grads)) return ONEBIT_ERR_ALIGN;
+    }
+    if (phase == 2) {
+        if (x == nullptr) return ONEBIT_ERR_ARG;
+        if (!aligned16(x)) return ONEBIT_ERR_ALIGN;
+    }
+    return ONEBIT_OK;
+}
+
+void dp_phase_done(onebit_adam_t h, int kind, int32_t phase) {
+    DpState& dp = h->dp;
+    dp.next_phase = (phase + 1) % 3;
+    dp.phase_kind = phase == 2 ? 0 : kind;
+}
+
+}  // namespace
+
+extern "C" {
+
+int onebit_dp_warmup_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
+                           float lr, void* stream) {
+    int rc = dp_phase_check(h, 1, phase, x, grads, lr);
+    if (rc != ONEBIT_OK) return rc;
+    if (h->geo.d > 0) {
+        rc = dp_warmup_phase(h, phase, x, grads, lr, phase > 0 ? kBarrierWait : 0,
+                             phase < 2 ? kBarrierSignal : 0, as_stream(stream));
+        if (rc != ONEBIT_OK) return rc;
+    }
+    dp_phase_done(h, 1, phase);
+    return ONEBIT_OK;
+}
+
+int onebit_dp_compressed_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
+                               float lr, void* stream) {
+    int rc = dp_phase_check(h, 2, phase, x, grads, lr);
+    if (rc != ONEBIT_OK) return rc;
+    if (h->geo.d > 0) {
+        rc = dp_compressed_phase(h, phase, x, grads, lr, phase > 0 ? kBarrierWait : 0,
+                                 phase < 2 ? kBarrierSignal : 0, as_stream(stream));
+        if (rc != ONEBIT_OK) return rc;
+    }
+    dp_phase_done(h, 2, phase);
+    if (phase == 2) {
+        if (h->tcount < h->tmax) ++h->tcount;
+        ++h->steps;
+        if (h->geo.d > 0) h->m_explicit = false;
+    }
+    return ONEBIT_OK;
 }
 
 int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* stream) {

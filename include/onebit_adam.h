@@ -19,7 +19,9 @@
  * Conventions (all calls):
  *   - Every pointer named *_dev or documented as device memory is a CUDA device pointer owned
  *     by the caller, 16-byte aligned, and must stay valid until the work queued on the stream
- *     has finished. The library never allocates device memory.
+ *     has finished. The library allocates no device memory, with one exception: the exchange
+ *     region of a data-parallel rank (onebit_dp_*), which other ranks map through CUDA IPC and
+ *     which therefore must be an allocation of its own.
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device work
  *     is queued on it asynchronously; argument errors are detected on the host and returned
  *     before anything is queued.
@@ -70,6 +72,10 @@ typedef enum {
 /* Device status flags (onebit_adam_status). */
 #define ONEBIT_FLAG_NAN_WORKER 1u /* some worker's x_w was NaN (its bit is 0) */
 #define ONEBIT_FLAG_NAN_SERVER 2u /* some server z was NaN */
+#define ONEBIT_FLAG_TIMEOUT 4u    /* a bounded wait gave up: a copy that did not land in the
+                                     server kernel, or a data-parallel barrier whose ranks did
+                                     not all arrive before the timeout; the step's results are
+                                     not valid */
 
 /*
  * Create a handle for d parameters, W workers, chunk length C ("1-bit Adam" index page,
@@ -240,6 +246,110 @@ int onebit_compress_static(const float* x, int64_t n, int64_t C, uint32_t* words
  * plumbing for the bounded waits.
  */
 int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* stream);
+
+/*
+ * ------------------------------------------------------------------------------------------
+ * Data-parallel ranks: the compressed allreduce across GPUs.
+ *
+ * The pages' compressed allreduce is a collective between machines ("1-bit Adam" index page,
+ * Abstract: communication over TCP is the bottleneck; LIT-278 note, "What the evidence does not
+ * cover": a custom collective). Here it runs between R GPUs of one NVLink/NVSwitch domain, one
+ * process (or, for emulation, one handle) per rank. Rank q holds W / R of the W workers
+ * (global workers q*W/R .. (q+1)*W/R - 1) and serves the chunks
+ * [q * nch / R, (q+1) * nch / R) (onebit_dp_chunk_range). A compressed step is:
+ *   phase 0  worker compression of the rank's workers; each plane word and scale is stored
+ *            directly into the receive buffers of the rank that serves its chunk; signal.
+ *   phase 1  wait for every rank; server average, residual and recompression of the rank's
+ *            chunks; each server plane word and scale is stored into every rank's copy; signal.
+ *   phase 2  wait for every rank; apply x -= lr * (m / (sqrt(v) + eps)) on all d elements.
+ * The warm-up likewise: phase 0 fp64 sums of the rank's gradients; phase 1 the rank's chunks
+ * read every rank's sums in rank order and write the Adam moments into every rank's m and v;
+ * phase 2 the x update. The results equal those of one single-GPU handle with all W workers
+ * (bit for bit in the compressed phase; in the warm-up whenever the fp64 sums of the gradients
+ * are exact, which their grouping by rank can otherwise change in the last bit).
+ *
+ * A rank's handle is used like a single-GPU one (workspace, bind, warm-up steps, freeze,
+ * compressed steps, state), with these additions and differences:
+ *   - onebit_dp_init instead of onebit_adam_init; W counts the workers of all ranks.
+ *   - onebit_adam_bind also allocates the exchange region (cudaMalloc; freed by
+ *     onebit_adam_destroy) and clears it. Every rank must then set its peers (onebit_dp_open_peer
+ *     from the peers' onebit_dp_ipc_handle, or onebit_dp_set_peer with addresses valid in this
+ *     process) and call onebit_dp_connect; all ranks must have finished connecting (and their
+ *     streams that work) before any rank takes a step -- a host barrier between connect and the
+ *     first step. Likewise before destroying a handle.
+ *   - Steps and freezes must be taken by all ranks in the same order. Each step contains two
+ *     barriers between the ranks (device-side flags, see ONEBIT_FLAG_TIMEOUT): a rank that never
+ *     arrives makes the others' waits give up after the timeout (onebit_dp_set_timeout, default
+ *     10 s), with ONEBIT_FLAG_TIMEOUT set in their status.
+ *   - State: ES is the server residual of the rank's own chunks (fp32[elements of those
+ *     chunks]); get_chunk_state(ES, k) needs a chunk k of the rank. EW, SW and BITSW cover the
+ *     rank's own workers (BITSW is rebuilt from the stored x_w, so after set_state(EW) it
+ *     reflects the residuals that were set). M, V, SS and BITSS cover all d elements and are the
+ *     same on every rank; set_state(M) and set_state(V) must be given the same values on every
+ *     rank, and set_state(ES) must be called by every rank (each with its own chunks).
+ *   - onebit_adam_info reports the rank's own worker count; kernel launches per compressed step
+ *     are 7 (two barrier launches).
+ * No rank's kernel ever waits on another rank's kernel unboundedly; a step that lost a rank
+ * still ends, with ONEBIT_FLAG_TIMEOUT set.
+ */
+
+#define ONEBIT_MAX_RANKS 8
+#define ONEBIT_IPC_HANDLE_BYTES 64
+
+/* Rank q's chunks [*k0, *k1) of nch chunks over R ranks (1 <= R <= 8). Host only. */
+int onebit_dp_chunk_range(int64_t nch, int32_t R, int32_t q, int64_t* k0, int64_t* k1);
+
+/*
+ * Create the handle of rank `rank` of R (1 <= R <= 8) for d parameters, W workers over all
+ * ranks (W % R == 0, W <= 256) and chunk length C; the other arguments and checks are those of
+ * onebit_adam_init. Host only.
+ */
+int onebit_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                   float beta2, float eps, int32_t R, int32_t rank);
+
+/*
+ * out[0..7] = R, rank, W over all ranks, first and end chunk of the rank's chunks, their first
+ * element, their element count, exchange region bytes.
+ */
+int onebit_dp_info(onebit_adam_t h, int64_t out[8]);
+
+/* Base address (device) and size of this rank's exchange region; bound handles only. */
+int onebit_dp_exchange(onebit_adam_t h, void** base, uint64_t* bytes);
+
+/* CUDA IPC handle (ONEBIT_IPC_HANDLE_BYTES bytes into out, host) of the exchange region. */
+int onebit_dp_ipc_handle(onebit_adam_t h, void* out);
+
+/*
+ * Map rank q's exchange region from its IPC handle (a different process on a peer GPU of the
+ * same node; peer access is enabled on demand). The mapping is released by
+ * onebit_adam_destroy or by setting the peer again.
+ */
+int onebit_dp_open_peer(onebit_adam_t h, int32_t q, const void* handle);
+
+/*
+ * Use `base` (device, 256-byte aligned, valid in this process: another handle's exchange
+ * region when several ranks are emulated in one process) as rank q's exchange region.
+ */
+int onebit_dp_set_peer(onebit_adam_t h, int32_t q, void* base);
+
+/* Build the rank's route from its peers and copy it to the device on `stream`. */
+int onebit_dp_connect(onebit_adam_t h, void* stream);
+
+/* Barrier timeout in microseconds (1 .. 3.6e9). */
+int onebit_dp_set_timeout(onebit_adam_t h, uint64_t timeout_us);
+
+/*
+ * One phase (0, 1, 2 in order; see above) of a warm-up or compressed step of this rank, for
+ * driving several emulated ranks from one thread: run phase p of every rank before phase p+1
+ * of any. Phase 0 reads grads ([W/R][d], device), phase 2 updates x (fp32[d], device); the
+ * other pointers may be NULL. Phases out of order return ONEBIT_ERR_PHASE. The whole-step
+ * entry points (onebit_adam_warmup_step, onebit_adam_compressed_step) run the three phases
+ * with one barrier launch between them and are what separate processes use.
+ */
+int onebit_dp_warmup_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
+                           float lr, void* stream);
+int onebit_dp_compressed_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
+                               float lr, void* stream);
 
 /* Static description of a status code. */
 const char* onebit_strerror(int32_t code);
