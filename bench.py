@@ -52,6 +52,9 @@ def parse_args():
                    help="replay the timed steps from a captured CUDA graph")
     p.add_argument("--scale-d", type=int, default=0,
                    help="run the workload's distributions on a smaller vector (profiling)")
+    p.add_argument("--dp", type=int, default=0,
+                   help="data-parallel ranks: with one process, R ranks emulated on this GPU; "
+                        "under torchrun, one rank per process (R = world size)")
     return p.parse_args()
 
 
@@ -399,6 +402,191 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_dp(args):
+    """The data-parallel step: R ranks, W / R workers each, rank q serving a 1/R share of the
+    chunks. One process: the R ranks are emulated as R handles on this GPU, stepped phase by
+    phase (the exchange then moves through this GPU's own memory); the single-GPU step of the
+    same workload is timed beside it. Under torchrun: one rank per process over CUDA IPC, the
+    value the whole job's params x workers / s (the W workers are fixed: strong scaling)."""
+    import torch
+    import torch.distributed as dist
+
+    import communication_compressed_optimizer_momentum_b200 as ob
+    from communication_compressed_optimizer_momentum_b200 import dp
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    R = world if world > 1 else args.dp
+    wl = get_workload(args.workload, args.scale_d)
+    if wl.W % R:
+        raise SystemExit("--dp %d: the workload's %d workers do not split over %d ranks"
+                         % (R, wl.W, R))
+    Wl = wl.W // R
+    dt = wls.torch_dtype(wl)
+    x0 = wls.torch_params(wl, dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
+        opt = dp.OneBitAdamRank(wl.d, wl.W, wl.C, R, rank, wl.beta1, wl.beta2, wl.eps,
+                                grad_dtype=dt, device=dev)
+        dp.connect_process_group(opt)
+        handles = [opt]
+        xs = [x0]
+        g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
+
+        def fill(phase, t):
+            wls.torch_fill_grads(wl, g, phase, t)
+            return [g[rank * Wl:(rank + 1) * Wl]]
+
+        def warm_step(gs):
+            opt.warmup_step(xs[0], gs[0], wl.lr)
+
+        def step(gs):
+            opt.step(xs[0], gs[0], wl.lr)
+
+        def freeze():
+            opt.freeze()
+        launches = 7
+    else:
+        em = dp.EmulatedRanks(wl.d, wl.W, wl.C, R, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
+                              device=dev)
+        handles = em.ranks
+        xs = [x0.clone() for _ in range(R)]
+        g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
+
+        def fill(phase, t):
+            wls.torch_fill_grads(wl, g, phase, t)
+            out = []
+            for r in range(R):
+                v = g[r * Wl:(r + 1) * Wl]
+                out.append(v if v.data_ptr() % 16 == 0 else v.clone())
+            return out
+
+        def warm_step(gs):
+            em.warmup_step(xs, gs, wl.lr)
+
+        def step(gs):
+            em.step(xs, gs, wl.lr)
+
+        def freeze():
+            em.freeze()
+        launches = 9 * R                  # phase by phase: a signal and a wait launch each
+    warm_ms = []
+    for t in range(wl.warmup_steps):
+        gs = fill(0, t)
+        w0 = torch.cuda.Event(enable_timing=True)
+        w1 = torch.cuda.Event(enable_timing=True)
+        w0.record()
+        warm_step(gs)
+        w1.record()
+        w1.synchronize()
+        warm_ms.append(w0.elapsed_time(w1))
+    freeze()
+    gs = fill(1, 1)
+    torch.cuda.synchronize()
+    for _ in range(max(args.warmup, 0)):
+        step(gs)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.5)
+    # per-kernel events of rank 0 (only meaningful when its launches are not interleaved with
+    # other emulated ranks': one process per rank, or a single rank)
+    per_kernel = world > 1 or R == 1
+    if per_kernel:
+        handles[0].timing(args.steps)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(gs)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    kernel_ms = None
+    if per_kernel:
+        kms, nrec = handles[0].timing_read()
+        handles[0].timing(0)
+        kernel_ms = {k: v / max(nrec, 1) for k, v in kms.items()}
+    time.sleep(0.3)
+    clocks = sampler.stop()
+    ms_max = max_over_ranks(ms, dev)
+    status = 0
+    for h in handles:
+        status |= h.status()
+    peak, peak_src = measured_hbm_peak()
+    n_gpu = max(world, 1)
+    step_bytes = wl.dp_algorithmic_bytes_per_param(R) * wl.d
+    achieved = step_bytes * args.steps / (ms_max / 1e3) / 1e9
+    single_ms = None
+    if world == 1:
+        # the single-GPU step of the same workload, same process, for comparison
+        for h in handles:
+            h.close()
+        del handles, xs
+        torch.cuda.empty_cache()
+        one = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
+                            device=dev)
+        x1 = x0.clone()
+        one.warmup_step(x1, g, wl.lr)
+        one.freeze()
+        for _ in range(max(args.warmup, 0)):
+            one.step(x1, g, wl.lr)
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            one.step(x1, g, wl.lr)
+        s1.record(stream)
+        torch.cuda.synchronize()
+        single_ms = s0.elapsed_time(s1) / args.steps
+        one.close()
+    else:
+        for h in handles:
+            h.close()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": whole_job_rate(wl.d * wl.W * args.steps, 1, ms_max),
+            "unit": UNIT, "n_gpus": n_gpu, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": dict(wls.describe(wl),
+                           parallelism=("dp%d" % R) if world > 1 else
+                           ("dp%d emulated on one GPU" % R),
+                           workers_per_rank=Wl,
+                           l2="inputs larger than L2; no flush"),
+            "achieved_hbm_gbs": achieved,
+            "pct_of_hbm_peak": 100.0 * achieved / (peak * n_gpu),
+            "algorithmic_bytes_per_step": step_bytes,
+            "roofline": {"bound": "hbm", "kernel": "whole data-parallel step",
+                         "achieved": achieved / n_gpu, "peak": peak, "peak_source": peak_src,
+                         "unit": "GB/s", "frac": achieved / n_gpu / peak, "traffic": None},
+            "single_gpu_ms_per_step": single_ms,
+            "rank0_kernel_ms_per_step": kernel_ms,
+            "warmup_phase": ({"steps": len(warm_ms),
+                              "ms_per_step": sum(warm_ms[1:]) / (len(warm_ms) - 1)}
+                             if len(warm_ms) > 1 else None),
+            "gpu_launches": launches * args.steps,
+            "clocks": clocks, "e2e": None, "cpu_baseline": None, "status_flags": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     """The oracle as it stands on the host cores, on a bounded sample of the same workload."""
     rank = int(os.environ.get("RANK", "0"))
@@ -440,6 +628,8 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.dp:
+        run_dp(args)
     else:
         run_ours(args)
 

@@ -283,22 +283,28 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
     }
     const float b1 = a.beta1, omb1 = a.omb1;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
-    uint32_t* bw0;
-    int64_t bld;
+    // DP: this block's destination row start and row length, kept in shared memory (the
+    // kernel runs at its register limit), and whether the destination is another rank's
+    __shared__ uint32_t* dp_bw0[1];
+    __shared__ int64_t dp_bld[1];
+    __shared__ int dp_remote[1];
     if constexpr (DP) {
-        const DpRoute* rt = a.route;
-        const int q = dp_owner(rt, k);
-        bld = rt->ldw[q];
-        bw0 = rt->planes[q] + (int64_t)rt->w0 * bld + ((base - rt->kb[q] * a.geo.C) >> 5);
-    } else {
-        bld = a.geo.ldw;
-        bw0 = a.bits_w + (base >> 5);
+        if (tid == 0) {
+            const DpRoute* rt = a.route;
+            const int q = dp_owner(rt, k);
+            dp_bld[0] = rt->ldw[q];
+            dp_bw0[0] = rt->planes[q] + (int64_t)rt->w0 * rt->ldw[q] +
+                        ((base - rt->kb[q] * a.geo.C) >> 5);
+            dp_remote[0] = q != rt->rank;
+        }
+        __syncthreads();
     }
     for (int w = 0; w < W; ++w) {
         const float sp = a.s_lazy[(int64_t)w * a.geo.nch + k];
         const GT* gw = g0 + (int64_t)w * a.geo.d;
         float* ew = a.ew + (int64_t)w * a.geo.ld + base;
-        uint32_t* bw = bw0 + (int64_t)w * bld;
+        uint32_t* bw = DP ? dp_bw0[0] + (int64_t)w * dp_bld[0]
+                          : a.bits_w + (int64_t)w * a.geo.ldw + (base >> 5);
         double ss = 0.0;
 #pragma unroll
         for (int it = 0; it < ITEMS; ++it) {
@@ -345,7 +351,11 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
         ss = warp_sum(ss);
         if (lane == 0) red_w[w * kWarps + warp] = ss;
     }
-    if constexpr (DP) __threadfence_system();  // peer stores before the rank's barrier signal
+    // stores into another rank's memory are complete at system scope before this rank's
+    // barrier signal (stores to this GPU's own memory are ordered by the kernel boundary)
+    if constexpr (DP) {
+        if (dp_remote[0]) __threadfence_system();
+    }
     __syncthreads();
     bool nan_seen = false;
     for (int w = tid; w < W; w += kThreads) {
@@ -414,19 +424,22 @@ __global__ void __launch_bounds__(kThreads) k_scales_dp(const double* part, int6
     const int64_t r = (int64_t)blockIdx.x * (kThreads / TPR) + threadIdx.x / TPR;
     const bool active = r < rows;
     const float s = row_scale<TPR>(part, r, active, nch, nseg, seg, C, d, red);
+    bool remote = false;
     if (active && threadIdx.x % TPR == 0) {
         lazy[r] = s;
         if constexpr (SERVER) {
             const int64_t kg = rt->kb[rt->rank] + r;
             for (int p = 0; p < rt->R; ++p) rt->S[p][kg] = s;
+            remote = rt->R > 1;
         } else {
             out[r] = s;
             const int64_t w = r / nch, k = r - w * nch;
             const int q = dp_owner(rt, k);
             rt->scales[q][(rt->w0 + w) * (rt->kb[q + 1] - rt->kb[q]) + (k - rt->kb[q])] = s;
+            remote = q != rt->rank;
         }
     }
-    __threadfence_system();
+    if (remote) __threadfence_system();  // peer stores before the barrier signal
 }
 
 // ------------------------------------------------------------------------------------------
@@ -616,8 +629,9 @@ __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stag
 }
 
 // BCAST (data-parallel ranks): the geometry is this rank's range of chunks, the plane rows are
-// the receive planes of all W workers, and every server plane word is stored into every rank's
-// server plane (the broadcast half of the compressed allreduce, to peer memory).
+// the receive planes of all W workers, bits_s points at this rank's first chunk in its own copy
+// of the server plane, and each block then stores its server words into every other rank's copy
+// (the broadcast half of the compressed allreduce, to peer memory).
 template <bool POW2, bool STAGE_RES, bool BCAST = false>
 __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     extern __shared__ __align__(16) unsigned char smem_srv[];
@@ -866,15 +880,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 uint32_t word = byte << (8 * (lane & 3));
                 word |= __shfl_xor_sync(kFull, word, 1);
                 word |= __shfl_xor_sync(kFull, word, 2);
-                if ((lane & 3) == 0 && nv > 0) {
-                    if constexpr (BCAST) {
-                        const DpRoute* rt = a.route;
-                        const int64_t gw = ((rt->kb[rt->rank] * a.geo.C) >> 5) + wbase + wd;
-                        for (int p = 0; p < rt->R; ++p) rt->bits_s[p][gw] = word;
-                    } else {
-                        a.bits_s[wbase + wd] = word;
-                    }
-                }
+                if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
             }
         }
         // everyone is done with this stage (or some thread's wait expired: then all leave,
@@ -891,7 +897,6 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             server_issue<STAGE_RES>(a, stages + (size_t)st * stage_words, wpad, &bars[st], c0,
                                     clen, j0 + t + nst);
     }
-    if constexpr (BCAST) __threadfence_system();  // peer stores before the barrier signal
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
@@ -899,6 +904,24 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
         const double tot = block_total(red);
         a.part_s[k * nsb + b] = tot;
         if (tot != tot) atomicOr(a.status, kNanServer);   // a NaN z makes the sum NaN
+    }
+    if constexpr (BCAST) {
+        // the block's server words, written to this rank's copy above (visible to the block
+        // after the barrier), go to every other rank's copy; word ranges of blocks are disjoint
+        // because chunks start on word boundaries
+        // (the block's element range is recomputed from k and b, so that nothing else has to
+        // stay live through the main loop)
+        const DpRoute* rt = a.route;
+        const int64_t e_lo = k * a.geo.C + b * (kSrvSegsPerBlock * kSegS);
+        const int64_t e_hi = min(min((k + 1) * a.geo.C, a.geo.d), e_lo + kSrvSegsPerBlock * kSegS);
+        const int64_t w_lo = e_lo >> 5, w_hi = (e_hi + 31) >> 5;
+        const int64_t gw0 = (rt->kb[rt->rank] * a.geo.C) >> 5;
+        for (int p = 0; p < rt->R; ++p) {
+            if (p == rt->rank) continue;
+            uint32_t* dst = rt->bits_s[p] + gw0;
+            for (int64_t i = w_lo + tid; i < w_hi; i += kThreads) dst[i] = __ldcg(a.bits_s + i);
+        }
+        if (rt->R > 1) __threadfence_system();  // peer stores before the barrier signal
     }
 }
 

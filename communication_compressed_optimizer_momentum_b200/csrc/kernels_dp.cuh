@@ -2,13 +2,15 @@
 // three warm-up kernels. The compressed step's kernels take their data-parallel form from
 // kernels.cuh (k_worker<..., DP>, k_server<..., BCAST>, k_scales_dp).
 //
-// Cross-rank ordering. A kernel that stores into peer memory ends every thread with a
-// system-scope fence; the barrier kernel that follows it on the stream then publishes the rank's
-// epoch into every rank's flag array with a system-scope release store, and waits (acquire
-// loads, bounded) until every rank's flag in its own array has reached the epoch. Kernels after
-// the barrier therefore see everything that every rank stored before its signal. Each wait has
-// a deadline: when it passes, the barrier sets the kWaitTimeout status bit and returns, so a
-// missing rank shows up as a status flag on the host instead of a hung GPU.
+// Cross-rank ordering. A thread that stored into another rank's memory ends with a
+// system-scope fence, so those stores are complete everywhere before its kernel finishes;
+// stores into the rank's own memory (read by peers later) are ordered by the kernel boundary.
+// The barrier kernel that follows on the stream then publishes the rank's epoch into every
+// rank's flag array with a system-scope release store, and waits (acquire loads, bounded) until
+// every rank's flag in its own array has reached the epoch. Kernels after the barrier
+// therefore see everything that every rank stored before its signal. Each wait has a deadline:
+// when it passes, the barrier sets the kWaitTimeout status bit and returns, so a missing rank
+// shows up as a status flag on the host instead of a hung GPU.
 #pragma once
 
 #include "kernels.cuh"
@@ -97,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 4) k_warmup_partial(const Geometry g
         for (int h = 0; h < EPT / 2; ++h)
             *reinterpret_cast<double2*>(dst + 2 * h) = make_double2(acc[2 * h], acc[2 * h + 1]);
     }
-    __threadfence_system();
 }
 
 struct WarmupDpArgs {
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kThreads) k_warmup_reduce(const WarmupDpArgs a
             st4(rt->v[p] + i, v);
         }
     }
-    __threadfence_system();
+    if (R > 1) __threadfence_system();  // peer stores before the barrier signal
 }
 
 struct WarmupApplyArgs {

@@ -454,8 +454,8 @@ int dp_compressed_phase(onebit_adam_s* h, int phase, float* x, const void* grads
         if (gs.d > 0) {
             uint32_t* planes = reinterpret_cast<uint32_t*>(dp.xch + dp.xl.planes);
             const float* rs = reinterpret_cast<const float*>(dp.xch + dp.xl.rscales);
-            ServerArgs sa{gs, planes, rs, h->es, h->S_lazy, nullptr, h->part_s, h->status,
-                          dp.route_dev};
+            ServerArgs sa{gs, planes, rs, h->es, h->S_lazy, h->bits_s + dp.e0 / 32, h->part_s,
+                          h->status, dp.route_dev};
             const size_t ssm = server_smem_bytes(gs.W, server_stages(gs.W, gs.nseg_s));
             server_kernel_dp(gs.W)<<<(unsigned)server_blocks(gs), kThreads, ssm, st>>>(sa);
             ONEBIT_CUDA(cudaGetLastError());

@@ -66,6 +66,14 @@ class Workload:
         are negligible and left out: W*(G + 8.25) + 20.375."""
         return self.W * (self.grad_bytes + 8.25) + 20.375
 
+    def dp_algorithmic_bytes_per_param(self, R: int) -> float:
+        """The same minimum for R data-parallel ranks together (W / R workers each; rank q
+        serves a 1/R share of the chunks; x, v and the server plane replicated): every rank's
+        worker pass reads the server plane to rebuild m (1/8 each), the server broadcasts its
+        plane to every rank (R/8 written) and every rank applies the step to its own x
+        (12.125 each). W*(G + 8.25) + 8 + 12.375*R, equal to the single-GPU figure at R = 1."""
+        return self.W * (self.grad_bytes + 8.25) + 8.0 + 12.375 * R
+
     def kernel_bytes_per_param(self) -> dict:
         """The same minimum, split by the three streaming kernels of the step."""
         G, W = self.grad_bytes, self.W

@@ -320,3 +320,26 @@ def test_bert_large_bucket_four_ranks():
     if free < 110e9:
         pytest.skip("needs about 110 GB of free device memory")
     run_against_single(wl, 4, warm=1, steps=2, check_every=False)
+
+
+def test_bench_dp_line():
+    """bench.py --dp 2 (two emulated ranks) prints one JSON line with the data-parallel step's
+    throughput, its roofline against the data-parallel byte count and the single-GPU step."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--dp", "2",
+                        "--workload", "smoke_1m", "--steps", "5", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["value"] > 0 and line["status_flags"] == 0
+    assert line["config"]["parallelism"] == "dp2 emulated on one GPU"
+    assert line["config"]["workers_per_rank"] == 2
+    assert line["gpu_launches"] == 9 * 2 * 5
+    assert line["single_gpu_ms_per_step"] > 0
+    wl = wls.WORKLOADS["smoke_1m"]
+    assert line["algorithmic_bytes_per_step"] == wl.dp_algorithmic_bytes_per_param(2) * wl.d
