@@ -37,16 +37,24 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
-// One warp. Thread q < R: signal stores `epoch` into rank q's flag of this rank; wait polls this
-// rank's flag of rank q until it reaches `epoch` (wrap-safe compare), for at most timeout_ns
-// and kBarrierPolls polls.
-__global__ void k_dp_barrier(const DpRoute* rt, uint32_t epoch, int mode, uint64_t timeout_ns,
+// One warp. The rank's barrier count lives in device memory (*epoch_p), so that a captured and
+// replayed step synchronizes like an eager one. Signal: the count goes up by one and thread
+// q < R stores it into rank q's flag of this rank. Wait: thread q < R polls this rank's flag of
+// rank q until it reaches the count (wrap-safe compare), for at most timeout_ns and
+// kBarrierPolls polls.
+__global__ void k_dp_barrier(const DpRoute* rt, uint32_t* epoch_p, int mode, uint64_t timeout_ns,
                              uint32_t* status) {
     const int t = threadIdx.x;
     const int R = rt->R, me = rt->rank;
-    if ((mode & kBarrierSignal) && t < R) {
-        __threadfence_system();
-        st_release_sys(rt->flags[t] + me, epoch);
+    uint32_t epoch = *epoch_p;
+    if (mode & kBarrierSignal) {
+        ++epoch;
+        __syncwarp();
+        if (t == 0) *epoch_p = epoch;
+        if (t < R) {
+            __threadfence_system();
+            st_release_sys(rt->flags[t] + me, epoch);
+        }
     }
     if (mode & kBarrierWait) {
         bool ok = true;

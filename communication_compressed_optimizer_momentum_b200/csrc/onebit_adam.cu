@@ -84,8 +84,8 @@ struct DpState {
     bool ipc[kMaxRanks] = {};          // peer mapped by CUDA IPC (closed at destroy)
     DpRoute route{};                   // host copy of the route
     DpRoute* route_dev = nullptr;      // device copy (in the workspace)
+    uint32_t* epoch_dev = nullptr;     // barriers signalled so far (device, after the route)
     bool connected = false;
-    uint32_t epoch = 0;                // barriers signalled so far
     int next_phase = 0;                // phase-by-phase driving: the phase expected next
     int phase_kind = 0;                // 0 none in progress, 1 warm-up, 2 compressed
     uint64_t timeout_ns = 10000000000ull;
@@ -133,7 +133,8 @@ Layout make_layout(const onebit_adam_s& h) {
         return at;
     };
     const uint64_t f = sizeof(float), u = sizeof(uint32_t);
-    L.route = take(dp ? sizeof(DpRoute) : 0);
+    // the route, then the rank's barrier count (kept across connects and freezes)
+    L.route = take(dp ? sizeof(DpRoute) + sizeof(uint32_t) : 0);
     L.m = take(dp ? 0 : g.ld * f);
     L.v = take(dp ? 0 : g.ld * f);
     L.es = take(gs.ld * f);
@@ -381,8 +382,7 @@ int launch_pack_rows(onebit_adam_s* h, int64_t i0, int64_t n, uint32_t* dst, cud
 
 int dp_barrier(onebit_adam_s* h, int mode, cudaStream_t st) {
     DpState& dp = h->dp;
-    if (mode & kBarrierSignal) ++dp.epoch;
-    k_dp_barrier<<<1, 32, 0, st>>>(dp.route_dev, dp.epoch, mode, dp.timeout_ns, h->status);
+    k_dp_barrier<<<1, 32, 0, st>>>(dp.route_dev, dp.epoch_dev, mode, dp.timeout_ns, h->status);
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }
@@ -581,8 +581,8 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
         h->S_out = reinterpret_cast<float*>(x + dp.xl.S);
         h->bits_w = nullptr;
         dp.route_dev = reinterpret_cast<DpRoute*>(b + L.route);
+        dp.epoch_dev = reinterpret_cast<uint32_t*>(b + L.route + sizeof(DpRoute));
         dp.connected = false;
-        dp.epoch = 0;
         dp.next_phase = 0;
         dp.phase_kind = 0;
         const int ssm = (int)server_smem_bytes(dp.Wg, server_stages(dp.Wg, dp.gs.nseg_s));

@@ -290,7 +290,8 @@ int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* strea
  *   - onebit_adam_info reports the rank's own worker count; kernel launches per compressed step
  *     are 7 (two barrier launches).
  * No rank's kernel ever waits on another rank's kernel unboundedly; a step that lost a rank
- * still ends, with ONEBIT_FLAG_TIMEOUT set.
+ * still ends, with ONEBIT_FLAG_TIMEOUT set. The barriers count in device memory, so a step (or
+ * a sequence of phases) can be captured in a CUDA graph and replayed like the single-GPU step.
  */
 
 #define ONEBIT_MAX_RANKS 8

@@ -311,6 +311,44 @@ def test_rank_checkpoint_resume():
     B.close()
 
 
+def test_graph_replay_of_rank_steps():
+    """A step of 2 emulated ranks captured in a CUDA graph and replayed equals eager steps: the
+    barriers count in device memory, so a replay synchronizes like a new step."""
+    wl, R = _wl(F32, 65_536, 4, 8192), 2
+    x = wls.torch_params(wl, DEV)
+    g = torch.empty((wl.W, wl.d), dtype=torch.float32, device=DEV)
+    eager = dp.EmulatedRanks(wl.d, wl.W, wl.C, R, device=DEV)
+    graphed = dp.EmulatedRanks(wl.d, wl.W, wl.C, R, device=DEV)
+    xe = [x.clone() for _ in range(R)]
+    xg = [x.clone() for _ in range(R)]
+    wls.torch_fill_grads(wl, g, 0, 0)
+    gs = _rank_grads(g, R)
+    for em, xs in ((eager, xe), (graphed, xg)):
+        em.warmup_step(xs, gs, wl.lr)
+        em.freeze()
+        em.step(xs, gs, wl.lr)          # the first step reads the explicit warm-up momentum
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        graphed.step(xg, gs, wl.lr)
+    torch.cuda.synchronize()
+    for t in range(4):
+        wls.torch_fill_grads(wl, g, 1, t + 2)    # new values in the captured buffers
+        gs2 = _rank_grads(g, R)
+        assert all(a.data_ptr() == b.data_ptr() for a, b in zip(gs, gs2))
+        eager.step(xe, gs, wl.lr)
+        graph.replay()
+        torch.cuda.synchronize()
+        for r in range(R):
+            assert _same(xe[r], xg[r]), "replay %d, rank %d" % (t, r)
+    assert eager.status() == 0 and graphed.status() == 0
+    del graph
+    eager.close()
+    graphed.close()
+
+
 @pytest.mark.slow
 def test_bert_large_bucket_four_ranks():
     """The BERT-Large bucket (333.6M parameters, 16 workers, bf16) over 4 emulated ranks equals
