@@ -3,8 +3,10 @@
 the ranks do (workers per rank, servers per chunk range, an exchange of plane slices and scales,
 a broadcast of the server plane) reproduces the single-process oracle step exactly.
 
-The last test uses the oracle only (the CUDA path needs a GPU); it pins the decomposition the
-data-parallel kernels rely on, with the library's own chunk ranges."""
+The decomposition test uses the oracle only (the CUDA path needs a GPU); it pins the
+decomposition the data-parallel kernels rely on, with the library's own chunk ranges. The last
+test runs ``connect_process_group`` on three gloo ranks with a stand-in for the rank handle and
+checks that every rank maps every other rank's exchange region from that rank's IPC handle."""
 import ctypes
 import datetime
 import os
@@ -204,3 +206,65 @@ def test_rank_decomposition_matches_the_single_process_step(lib, world):
         assert np.array_equal(mr.view(np.uint32), m.view(np.uint32))
         assert np.array_equal(ewr, e_w[rank * Wl:(rank + 1) * Wl])
         assert np.array_equal(esr, e_s[e0:e1])
+
+
+# ----------------------------------------------------------------------------------------------
+# connect_process_group's exchange of IPC handles, on gloo ranks with a stand-in handle
+
+
+class _StubRank:
+    """Records what connect_process_group asks of a rank's handle (no GPU needed)."""
+
+    def __init__(self, R, rank):
+        self.R, self.rank = R, rank
+        self.opened = {}
+        self.connected = False
+
+    def ipc_handle(self):
+        return bytes([self.rank]) * 64
+
+    def open_peer(self, q, handle):
+        self.opened[q] = handle
+
+    def connect(self, stream=None):
+        self.connected = True
+
+
+def _connect_main(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    from communication_compressed_optimizer_momentum_b200 import dp
+    torch.cuda.synchronize = lambda *a, **k: None       # no device in this test
+    stub = _StubRank(world, rank)
+    dp.connect_process_group(stub)
+    bad = _StubRank(world + 1, rank)
+    try:
+        dp.connect_process_group(bad)
+        mismatch = False
+    except ValueError:
+        mismatch = True
+    q.put((rank, sorted(stub.opened.items()), stub.connected, mismatch))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_connect_process_group_routes_every_peer_handle(lib):
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = [ctx.Process(target=_connect_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, opened, connected, mismatch in out:
+        assert connected and mismatch
+        assert opened == [(p, bytes([p]) * 64) for p in range(world) if p != rank]
