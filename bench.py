@@ -420,7 +420,10 @@ def run_dp(args):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    R = world if world > 1 else args.dp
+    # under torchrun (even with one process) each process is one rank over a process group;
+    # a plain process emulates args.dp ranks on its GPU
+    real = world > 1 or "LOCAL_RANK" in os.environ
+    R = world if real else args.dp
     wl = get_workload(args.workload, args.scale_d)
     if wl.W % R:
         raise SystemExit("--dp %d: the workload's %d workers do not split over %d ranks"
@@ -428,7 +431,7 @@ def run_dp(args):
     Wl = wl.W // R
     dt = wls.torch_dtype(wl)
     x0 = wls.torch_params(wl, dev)
-    if world > 1:
+    if real:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
         opt = dp.OneBitAdamRank(wl.d, wl.W, wl.C, R, rank, wl.beta1, wl.beta2, wl.eps,
@@ -440,7 +443,8 @@ def run_dp(args):
 
         def fill(phase, t):
             wls.torch_fill_grads(wl, g, phase, t)
-            return [g[rank * Wl:(rank + 1) * Wl]]
+            v = g[rank * Wl:(rank + 1) * Wl]
+            return [v if v.data_ptr() % 16 == 0 else v.clone()]
 
         def warm_step(gs):
             opt.warmup_step(xs[0], gs[0], wl.lr)
@@ -497,12 +501,12 @@ def run_dp(args):
     time.sleep(0.5)
     # per-kernel events of rank 0 (only meaningful when its launches are not interleaved with
     # other emulated ranks': one process per rank, or a single rank)
-    per_kernel = world > 1 or R == 1
+    per_kernel = real or R == 1
     if per_kernel:
         handles[0].timing(args.steps)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
+    if real:
         dist.barrier()
     torch.cuda.synchronize()
     t0.record(stream)
@@ -510,7 +514,7 @@ def run_dp(args):
         step(gs)
     t1.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
+    if real:
         dist.barrier()
     ms = t0.elapsed_time(t1)
     kernel_ms = None
@@ -560,10 +564,10 @@ def run_dp(args):
             "metric": METRIC, "value": whole_job_rate(wl.d * wl.W * args.steps, 1, ms_max),
             "unit": UNIT, "n_gpus": n_gpu, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "f32",
+            "scaling": "strong" if real else "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": dict(wls.describe(wl),
-                           parallelism=("dp%d" % R) if world > 1 else
+                           parallelism=("dp%d" % R) if real else
                            ("dp%d emulated on one GPU" % R),
                            workers_per_rank=Wl,
                            l2="inputs larger than L2; no flush"),
@@ -582,7 +586,7 @@ def run_dp(args):
             "clocks": clocks, "e2e": None, "cpu_baseline": None, "status_flags": status,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if real:
         dist.barrier()
         dist.destroy_process_group()
 

@@ -381,3 +381,59 @@ def test_bench_dp_line():
     assert line["single_gpu_ms_per_step"] > 0
     wl = wls.WORKLOADS["smoke_1m"]
     assert line["algorithmic_bytes_per_step"] == wl.dp_algorithmic_bytes_per_param(2) * wl.d
+
+
+def test_bench_dp_under_torchrun_one_process():
+    """bench.py --dp under torchrun takes the one-process-per-rank path (NCCL process group,
+    IPC handle exchange, whole-step entry points with one barrier launch each), here with one
+    rank on this GPU."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+                        "--nproc-per-node", "1", "--master-addr", "127.0.0.1",
+                        "--master-port", str(port), os.path.join(root, "bench.py"), "--dp", "1",
+                        "--workload", "smoke_1m", "--steps", "5", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["config"]["parallelism"] == "dp1" and line["scaling"] == "strong"
+    assert line["gpu_launches"] == 7 * 5 and line["status_flags"] == 0
+    assert line["value"] > 0 and line["rank0_kernel_ms_per_step"]["worker"] > 0
+
+
+def test_host_buffer_step_of_a_rank():
+    """onebit_adam_compressed_step_host on a one-rank handle (upload, step with its barriers,
+    read-back of x) gives the single-GPU handle's x."""
+    wl = _wl(F32, 50_000, 4, 8192)
+    x1 = wls.torch_params(wl, DEV)
+    x2 = x1.clone()
+    g = torch.empty((wl.W, wl.d), dtype=torch.float32, device=DEV)
+    single = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, device=DEV)
+    opt = _fused_rank(wl)
+    opt.connect()
+    wls.torch_fill_grads(wl, g, 0, 0)
+    single.warmup_step(x1, g, wl.lr)
+    opt.warmup_step(x2, g, wl.lr)
+    single.freeze()
+    opt.freeze()
+    g_host = torch.empty((wl.W, wl.d), dtype=torch.float32, pin_memory=True)
+    x_host = torch.empty(wl.d, dtype=torch.float32, pin_memory=True)
+    g_dev = torch.empty_like(g)
+    for t in range(1, 4):
+        wls.torch_fill_grads(wl, g, 1, t)
+        g_host.copy_(g)
+        single.step(x1, g, wl.lr)
+        opt.step_host(x2, g_dev, g_host, x_host, wl.lr)
+        opt.host_wait()
+        torch.cuda.synchronize()
+        assert torch.equal(x_host.view(torch.int32), x1.cpu().view(torch.int32)), t
+    assert opt.status() == 0
+    opt.close()
+    single.close()
