@@ -437,3 +437,16 @@ def test_host_buffer_step_of_a_rank():
     assert opt.status() == 0
     opt.close()
     single.close()
+
+
+def test_empty_vector_ranks():
+    """d = 0: every phase and step of the ranks is a no-op that succeeds."""
+    em = dp.EmulatedRanks(0, 4, 64, 2, device=DEV)
+    xs = [torch.empty(0, device=DEV) for _ in range(2)]
+    gs = [torch.empty((2, 0), device=DEV) for _ in range(2)]
+    em.warmup_step(xs, gs, 1e-3)
+    em.freeze()
+    em.step(xs, gs, 1e-3)
+    assert em.status() == 0
+    assert all(o.info()["steps"] == 1 for o in em.ranks)
+    em.close()
