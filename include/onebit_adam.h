@@ -297,55 +297,78 @@ int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* strea
 #define ONEBIT_MAX_RANKS 8
 #define ONEBIT_IPC_HANDLE_BYTES 64
 
-/* Rank q's chunks [*k0, *k1) of nch chunks over R ranks (1 <= R <= 8). Host only. */
+/*
+ * Rank q's chunks [*k0, *k1) of nch chunks over R ranks (1 <= R <= 8): contiguous, in rank
+ * order, sizes differing by at most one. Host only. ONEBIT_ERR_ARG for nch < 0, R or q out of
+ * range, or a NULL output.
+ */
 int onebit_dp_chunk_range(int64_t nch, int32_t R, int32_t q, int64_t* k0, int64_t* k1);
 
 /*
  * Create the handle of rank `rank` of R (1 <= R <= 8) for d parameters, W workers over all
  * ranks (W % R == 0, W <= 256) and chunk length C; the other arguments and checks are those of
- * onebit_adam_init. Host only.
+ * onebit_adam_init. Host only. ONEBIT_ERR_ARG for R, rank or W out of range or W % R != 0
+ * (*out is then NULL).
  */
 int onebit_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
                    float beta2, float eps, int32_t R, int32_t rank);
 
 /*
  * out[0..7] = R, rank, W over all ranks, first and end chunk of the rank's chunks, their first
- * element, their element count, exchange region bytes.
+ * element, their element count, exchange region bytes. ONEBIT_ERR_ARG for a single-GPU handle.
  */
 int onebit_dp_info(onebit_adam_t h, int64_t out[8]);
 
-/* Base address (device) and size of this rank's exchange region; bound handles only. */
+/*
+ * Base address (device) and size of this rank's exchange region, which the handle owns.
+ * ONEBIT_ERR_PHASE before onebit_adam_bind.
+ */
 int onebit_dp_exchange(onebit_adam_t h, void** base, uint64_t* bytes);
 
-/* CUDA IPC handle (ONEBIT_IPC_HANDLE_BYTES bytes into out, host) of the exchange region. */
+/*
+ * CUDA IPC handle (ONEBIT_IPC_HANDLE_BYTES bytes into out, host memory) of the exchange region,
+ * for the other ranks' onebit_dp_open_peer. ONEBIT_ERR_PHASE before onebit_adam_bind,
+ * ONEBIT_ERR_CUDA if the runtime refuses.
+ */
 int onebit_dp_ipc_handle(onebit_adam_t h, void* out);
 
 /*
  * Map rank q's exchange region from its IPC handle (a different process on a peer GPU of the
- * same node; peer access is enabled on demand). The mapping is released by
- * onebit_adam_destroy or by setting the peer again.
+ * same node; peer access is enabled on demand; call with this rank's device current). The
+ * handle owns the mapping and releases it in onebit_adam_destroy or when the peer is set
+ * again. ONEBIT_ERR_ARG for q out of range or q == rank, ONEBIT_ERR_CUDA if the mapping fails.
+ * Invalidates the route until the next onebit_dp_connect.
  */
 int onebit_dp_open_peer(onebit_adam_t h, int32_t q, const void* handle);
 
 /*
  * Use `base` (device, 256-byte aligned, valid in this process: another handle's exchange
- * region when several ranks are emulated in one process) as rank q's exchange region.
+ * region when several ranks are emulated in one process) as rank q's exchange region; the
+ * caller keeps it alive. ONEBIT_ERR_ARG for q out of range, q == rank or NULL,
+ * ONEBIT_ERR_ALIGN for a misaligned base. Invalidates the route until onebit_dp_connect.
  */
 int onebit_dp_set_peer(onebit_adam_t h, int32_t q, void* base);
 
-/* Build the rank's route from its peers and copy it to the device on `stream`. */
+/*
+ * Build the rank's route (every rank's buffer addresses) from its peers and copy it to the
+ * device on `stream`. ONEBIT_ERR_PHASE before onebit_adam_bind or while a peer is not set.
+ */
 int onebit_dp_connect(onebit_adam_t h, void* stream);
 
-/* Barrier timeout in microseconds (1 .. 3.6e9). */
+/* Barrier timeout in microseconds (1 .. 3.6e9; ONEBIT_ERR_ARG otherwise). Default 10 s. */
 int onebit_dp_set_timeout(onebit_adam_t h, uint64_t timeout_us);
 
 /*
  * One phase (0, 1, 2 in order; see above) of a warm-up or compressed step of this rank, for
  * driving several emulated ranks from one thread: run phase p of every rank before phase p+1
  * of any. Phase 0 reads grads ([W/R][d], device), phase 2 updates x (fp32[d], device); the
- * other pointers may be NULL. Phases out of order return ONEBIT_ERR_PHASE. The whole-step
- * entry points (onebit_adam_warmup_step, onebit_adam_compressed_step) run the three phases
- * with one barrier launch between them and are what separate processes use.
+ * other pointers may be NULL. ONEBIT_ERR_PHASE for a phase out of order, an unconnected rank,
+ * or the wrong phase of the method (warm-up after the freeze, compressed before it);
+ * ONEBIT_ERR_ARG for phase > 2, a single-GPU handle, a non-finite lr or a NULL pointer that the
+ * phase reads; ONEBIT_ERR_ALIGN for a pointer that is not 16-byte aligned. While a step is
+ * driven phase by phase, the freeze and the whole-step entry points return ONEBIT_ERR_PHASE.
+ * The whole-step entry points (onebit_adam_warmup_step, onebit_adam_compressed_step) run the
+ * three phases with one barrier launch between them and are what separate processes use.
  */
 int onebit_dp_warmup_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
                            float lr, void* stream);
