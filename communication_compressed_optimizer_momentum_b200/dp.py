@@ -147,6 +147,11 @@ class EmulatedRanks:
         raise IndexError(k)
 
     def close(self) -> None:
+        """Release every rank together (a rank must not step once a peer's exchange region is
+        freed); waits for the device first."""
+        import torch
+        if self.ranks:
+            torch.cuda.synchronize()
         for opt in self.ranks:
             opt.close()
         self.ranks = []

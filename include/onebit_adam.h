@@ -276,7 +276,9 @@ int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* strea
  *     from the peers' onebit_dp_ipc_handle, or onebit_dp_set_peer with addresses valid in this
  *     process) and call onebit_dp_connect; all ranks must have finished connecting (and their
  *     streams that work) before any rank takes a step -- a host barrier between connect and the
- *     first step. Likewise before destroying a handle.
+ *     first step. Likewise before destroying a handle: every rank's work must have finished
+ *     first, and once any rank's handle is destroyed (its exchange region freed) the others
+ *     must take no further step or phase.
  *   - Steps and freezes must be taken by all ranks in the same order. Each step contains two
  *     barriers between the ranks (device-side flags, see ONEBIT_FLAG_TIMEOUT): a rank that never
  *     arrives makes the others' waits give up after the timeout (onebit_dp_set_timeout, default
