@@ -1,4 +1,4 @@
-"""Two data-parallel ranks as two processes, connected through CUDA IPC.
+"""Data-parallel ranks as separate processes (two and three), connected through CUDA IPC.
 
 Each rank is its own process with its own CUDA context; the exchange regions are mapped across
 the processes with onebit_dp_ipc_handle / onebit_dp_open_peer, so the worker, server and warm-up
@@ -22,20 +22,20 @@ from gpu_helpers import DEV
 
 pytestmark = pytest.mark.gpu
 
-D, W, C, R = 20_000, 4, 2048, 2
+D, C = 20_000, 2048
 B1, B2, EPS, LR = 0.9, 0.999, 1e-8, 1e-3
 WARM, STEPS = 2, 3
 
 
-def _inputs():
-    rng = np.random.default_rng(4242)
+def _inputs(W):
+    rng = np.random.default_rng(4242 + W)
     x0 = rng.uniform(-0.05, 0.05, D).astype(np.float32)
     gw = [(rng.standard_normal((W, D)) * 1e-2).astype(np.float32) for _ in range(WARM)]
     gc = [(rng.standard_normal((W, D)) * 1e-2).astype(np.float32) for _ in range(STEPS)]
     return x0, gw, gc
 
 
-def _rank(rank, cmd, out):
+def _rank(rank, R, W, cmd, out):
     """Child process: one rank. Runs the commands the test host sends, one at a time."""
     import sys
     import os
@@ -44,7 +44,7 @@ def _rank(rank, cmd, out):
     from communication_compressed_optimizer_momentum_b200 import dp
     try:
         torch.cuda.set_device(0)
-        x0, gw, gc = _inputs()
+        x0, gw, gc = _inputs(W)
         Wl = W // R
         opt = dp.OneBitAdamRank(D, W, C, R, rank, B1, B2, EPS, device="cuda:0")
         opt.set_timeout_us(2_000_000)
@@ -55,7 +55,8 @@ def _rank(rank, cmd, out):
             msg = cmd.get(timeout=300)
             kind = msg[0]
             if kind == "open":
-                opt.open_peer(msg[1], msg[2])
+                for q, h in msg[1]:
+                    opt.open_peer(q, h)
                 opt.connect()
             elif kind == "warm":
                 opt.warmup_phase(msg[2], x, mine(gw[msg[1]]), LR)
@@ -85,17 +86,19 @@ def _expect(out, what, rank):
     return msg
 
 
-def test_two_processes_over_ipc_match_the_single_handle():
+@pytest.mark.parametrize("R", [2, 3])
+def test_rank_processes_over_ipc_match_the_single_handle(R):
+    W = 2 * R
     ctx = pymp.get_context("spawn")
     cmds = [ctx.Queue() for _ in range(R)]
     outs = [ctx.Queue() for _ in range(R)]
-    procs = [ctx.Process(target=_rank, args=(r, cmds[r], outs[r])) for r in range(R)]
+    procs = [ctx.Process(target=_rank, args=(r, R, W, cmds[r], outs[r])) for r in range(R)]
     for p in procs:
         p.start()
     try:
         handles = [_expect(outs[r], "handle", r)[2] for r in range(R)]
         for r in range(R):
-            cmds[r].put(("open", 1 - r, handles[1 - r]))
+            cmds[r].put(("open", [(q, handles[q]) for q in range(R) if q != r]))
             _expect(outs[r], "done", r)
 
         def run(kind, t):
@@ -117,7 +120,7 @@ def test_two_processes_over_ipc_match_the_single_handle():
             msg = _expect(outs[r], "result", r)
             assert msg[3] == 0, "rank %d status flags %d" % (r, msg[3])
             xs.append(msg[2])
-        for r in (1, 0):                    # the importer lets go before the exporter frees
+        for r in reversed(range(R)):        # every rank waits on the device, then lets go
             cmds[r].put(("close",))
             _expect(outs[r], "closed", r)
     finally:
@@ -128,7 +131,7 @@ def test_two_processes_over_ipc_match_the_single_handle():
     for p in procs:
         assert p.exitcode == 0
 
-    x0, gw, gc = _inputs()
+    x0, gw, gc = _inputs(W)
     x = torch.from_numpy(x0).to(DEV)
     single = ob.OneBitAdam(D, W, C, B1, B2, EPS, device=DEV)
     for g in gw:
