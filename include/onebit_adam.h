@@ -357,7 +357,11 @@ int onebit_dp_set_peer(onebit_adam_t h, int32_t q, void* base);
  */
 int onebit_dp_connect(onebit_adam_t h, void* stream);
 
-/* Barrier timeout in microseconds (1 .. 3.6e9; ONEBIT_ERR_ARG otherwise). Default 10 s. */
+/*
+ * Barrier timeout in microseconds (1 .. 3.6e9; ONEBIT_ERR_ARG otherwise). Default 10 s. A wait
+ * also ends after 2^28 polls (each followed by a nanosleep of about 256 ns), whichever comes
+ * first.
+ */
 int onebit_dp_set_timeout(onebit_adam_t h, uint64_t timeout_us);
 
 /*
