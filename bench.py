@@ -579,6 +579,11 @@ def run_dp(args):
                          "unit": "GB/s", "frac": achieved / n_gpu / peak, "traffic": None},
             "single_gpu_ms_per_step": single_ms,
             "rank0_kernel_ms_per_step": kernel_ms,
+            # what crosses NVLink between real ranks (here it stays in this GPU's memory when
+            # the ranks are emulated), against the measured 770 GB/s peer copy bandwidth
+            "nvlink": {"bytes_per_rank_per_step": wl.dp_nvlink_bytes_per_rank(R),
+                       "ms_at_770_gbs": wl.dp_nvlink_bytes_per_rank(R) / 770e9 * 1e3,
+                       "hbm_ms_per_rank_at_peak": step_bytes / R / (peak * 1e9) * 1e3},
             "warmup_phase": ({"steps": len(warm_ms),
                               "ms_per_step": sum(warm_ms[1:]) / (len(warm_ms) - 1)}
                              if len(warm_ms) > 1 else None),

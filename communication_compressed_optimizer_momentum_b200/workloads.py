@@ -74,6 +74,13 @@ class Workload:
         (12.125 each). W*(G + 8.25) + 8 + 12.375*R, equal to the single-GPU figure at R = 1."""
         return self.W * (self.grad_bytes + 8.25) + 8.0 + 12.375 * R
 
+    def dp_nvlink_bytes_per_rank(self, R: int) -> float:
+        """Bytes one of R data-parallel ranks stores into other ranks' memory per compressed
+        step, on average over the ranks: the sign words of its W / R workers for the chunks the
+        other ranks serve, and its share of the server plane for every other rank (per-chunk
+        scales are negligible). (W / R + 1) * d * (R - 1) / (8 R)."""
+        return (self.W / R + 1) * self.d * (R - 1) / (8.0 * R)
+
     def kernel_bytes_per_param(self) -> dict:
         """The same minimum, split by the three streaming kernels of the step."""
         G, W = self.grad_bytes, self.W

@@ -381,6 +381,7 @@ def test_bench_dp_line():
     assert line["single_gpu_ms_per_step"] > 0
     wl = wls.WORKLOADS["smoke_1m"]
     assert line["algorithmic_bytes_per_step"] == wl.dp_algorithmic_bytes_per_param(2) * wl.d
+    assert line["nvlink"]["bytes_per_rank_per_step"] == wl.dp_nvlink_bytes_per_rank(2)
 
 
 def test_bench_dp_under_torchrun_one_process():

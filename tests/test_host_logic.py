@@ -46,6 +46,18 @@ def test_algorithmic_bytes_split_by_kernel():
     assert wls.WORKLOADS["bert_large_bucket"].algorithmic_bytes_per_param() == 184.375
 
 
+def test_data_parallel_byte_counts():
+    """One rank is the single-GPU step; each extra rank adds one apply pass (x, v and the server
+    plane read, x written) and a copy of the server plane; the NVLink bytes are the sign words
+    and server-plane shares that leave a rank."""
+    for w in list(wls.WORKLOADS.values()) + [wls.sweep_workload(64, None)]:
+        assert w.dp_algorithmic_bytes_per_param(1) == w.algorithmic_bytes_per_param()
+        assert w.dp_algorithmic_bytes_per_param(4) - w.dp_algorithmic_bytes_per_param(3) == 12.375
+        assert w.dp_nvlink_bytes_per_rank(1) == 0
+    bl = wls.WORKLOADS["bert_large_bucket"]                     # W = 16, 8 ranks of 2 workers
+    assert bl.dp_nvlink_bytes_per_rank(8) == pytest.approx(3 * bl.d * 7 / 64)
+
+
 def test_scaled_workload_keeps_segment_proportions():
     wl = wls.scaled(wls.WORKLOADS["bert_base_bucket"], 1 << 20)
     assert wl.d == 1 << 20 and sum(wl.layer_sizes) == wl.d and len(wl.layer_sizes) == 13
