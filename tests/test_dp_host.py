@@ -268,3 +268,17 @@ def test_connect_process_group_routes_every_peer_handle(lib):
     for rank, opened, connected, mismatch in out:
         assert connected and mismatch
         assert opened == [(p, bytes([p]) * 64) for p in range(world) if p != rank]
+
+
+def test_python_rank_classes_check_arguments_on_the_host(lib):
+    """Bad rank counts are refused before any device memory is touched."""
+    from communication_compressed_optimizer_momentum_b200 import dp
+    with pytest.raises(ValueError):
+        dp.EmulatedRanks(1000, 8, 256, 9, device="cpu")
+    with pytest.raises(ValueError):
+        dp.EmulatedRanks(1000, 8, 256, 0, device="cpu")
+    with pytest.raises(ob.OneBitError) as e:
+        dp.OneBitAdamRank(1000, 6, 256, 4, 0, device="cpu")     # 6 workers over 4 ranks
+    assert e.value.code == -1
+    with pytest.raises(ob.OneBitError):
+        dp.OneBitAdamRank(1000, 8, 256, 2, 2, device="cpu")     # no rank 2 of 2
