@@ -248,23 +248,61 @@ def onebit_selftest_bounded_wait(polls: int, stream=None) -> bool:
     return int(flag.item()) == 1
 
 
+def _device_vector(t, dtype, min_numel: int, name: str, device=None):
+    """Check that ``t`` is a contiguous CUDA tensor of ``dtype`` with at least ``min_numel``
+    elements (on ``device`` when given) before its pointer goes to the library, which trusts
+    the sizes it is given."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device.type != "cuda":
+        raise ValueError("%s must be a CUDA tensor, got device %s" % (name, t.device))
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.numel() < min_numel:
+        raise ValueError("%s holds %d elements, needs at least %d" % (name, t.numel(), min_numel))
+
+
+def _chunk_length(C: int) -> int:
+    C = int(C)
+    if C <= 0 or C % 32 != 0:
+        raise ValueError("chunk length C must be a positive multiple of 32, got %d" % C)
+    return C
+
+
 def onebit_pack(x, words=None, stream=None):
     """Sign-pack a contiguous float32 CUDA tensor into int32 words (LSB-first)."""
     import torch
+    _device_vector(x, torch.float32, 0, "x")
     n = x.numel()
     if words is None:
         words = torch.empty((n + 31) // 32, dtype=torch.int32, device=x.device)
-    _check(_abi.lib().onebit_pack(_ptr(x), n, _ptr(words), _stream(stream)), "onebit_pack")
+    _device_vector(words, torch.int32, (n + 31) // 32, "words", x.device)
+    with torch.cuda.device(x.device):
+        st = _stream(stream if stream is not None else torch.cuda.current_stream(x.device))
+        _check(_abi.lib().onebit_pack(_ptr(x), n, _ptr(words), st), "onebit_pack")
     return words
 
 
 def onebit_unpack(words, scales, n: int, C: int, out=None, stream=None):
-    """Decompress packed words with per-chunk scales into a float32 CUDA tensor."""
+    """Decompress packed words with per-chunk scales into a float32 CUDA tensor (C >= 1)."""
     import torch
+    n, C = int(n), int(C)
+    if n < 0 or C < 1:
+        raise ValueError("need n >= 0 and C >= 1, got n=%d C=%d" % (n, C))
+    _device_vector(words, torch.int32, (n + 31) // 32, "words")
+    _device_vector(scales, torch.float32, (n + C - 1) // C, "scales", words.device)
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=words.device)
-    _check(_abi.lib().onebit_unpack(_ptr(words), _ptr(scales), n, C, _ptr(out), _stream(stream)),
-           "onebit_unpack")
+    _device_vector(out, torch.float32, n, "out", words.device)
+    with torch.cuda.device(words.device):
+        st = _stream(stream if stream is not None else torch.cuda.current_stream(words.device))
+        _check(_abi.lib().onebit_unpack(_ptr(words), _ptr(scales), n, C, _ptr(out), st),
+               "onebit_unpack")
     return out
 
 
@@ -274,13 +312,19 @@ def onebit_compress_static(x, C: int, words=None, scales=None, stream=None):
     that cannot allocate, pass preallocated ``words`` (int32, ceil(n/32)) and ``scales``
     (float32, ceil(n/C)); the defaults here allocate them with torch for convenience."""
     import torch
+    C = _chunk_length(C)
+    _device_vector(x, torch.float32, 0, "x")
     n = x.numel()
     if words is None:
         words = torch.empty((n + 31) // 32, dtype=torch.int32, device=x.device)
     if scales is None:
         scales = torch.empty((n + C - 1) // C, dtype=torch.float32, device=x.device)
-    _check(_abi.lib().onebit_compress_static(_ptr(x), n, C, _ptr(words), _ptr(scales),
-                                             _stream(stream)), "onebit_compress_static")
+    _device_vector(words, torch.int32, (n + 31) // 32, "words", x.device)
+    _device_vector(scales, torch.float32, (n + C - 1) // C, "scales", x.device)
+    with torch.cuda.device(x.device):
+        st = _stream(stream if stream is not None else torch.cuda.current_stream(x.device))
+        _check(_abi.lib().onebit_compress_static(_ptr(x), n, C, _ptr(words), _ptr(scales), st),
+               "onebit_compress_static")
     return words, scales
 
 

@@ -229,7 +229,9 @@ int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t
  *   onebit_last_error(), before any device work.
  *   C >= 32, C % 32 == 0 (ONEBIT_ERR_ALIGN otherwise); x 16-byte aligned; n = 0 is a no-op.
  *   The first call on each device looks up the array's device address (with that device
- *   current) and caches it; make that first call before any stream capture.
+ *   current) and caches it by device ordinal for the life of the process; make that first
+ *   call before any stream capture. A device reset (cudaDeviceReset, or a reset of the primary
+ *   context) invalidates the cached address: do not call this entry point after one.
  *   All calls share the one array and it keeps the last call's contents; each call writes every
  *   slot it reads before reading it. Calls whose work overlaps on the GPU (for example on two
  *   streams at once) race on the array and must be ordered by the caller.

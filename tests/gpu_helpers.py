@@ -67,6 +67,12 @@ class StepReport:
     s_total: int = 0
     S_exact: int = 0
     S_total: int = 0
+    ew_exact: int = 0
+    ew_total: int = 0
+    es_exact: int = 0
+    es_total: int = 0
+    m_exact: int = 0
+    m_total: int = 0
     max_rel_x: float = 0.0
     inexact_chunks: int = 0
 
@@ -102,6 +108,9 @@ def check_compressed_step(pre: Dict[str, np.ndarray], g: np.ndarray, post: Dict[
     d_ew = np.abs(post["e_w"] - e_w)
     bad = (d_ew > RTOL * s_el) & ~tie_w
     assert not bad.any(), "worker residuals differ at %d elements" % bad.sum()
+    # the tolerance is the assertion; how many non-tie values matched bit for bit is reported
+    rep.ew_exact = int(((post["e_w"].view(np.uint32) == e_w.view(np.uint32)) & ~tie_w).sum())
+    rep.ew_total = int((~tie_w).sum())
 
     S_el = expand(out["S"], C, n)
     S_g = post["S"].reshape(out["S"].shape)
@@ -118,6 +127,9 @@ def check_compressed_step(pre: Dict[str, np.ndarray], g: np.ndarray, post: Dict[
     assert not bad.any(), "server residuals differ at %d elements" % bad.sum()
     bad = (np.abs(post["m"] - m) > RTOL * S_el) & ~tie_s
     assert not bad.any(), "momentum differs at %d elements" % bad.sum()
+    rep.es_exact = int(((post["e_s"].view(np.uint32) == e_s.view(np.uint32)) & ~tie_s).sum())
+    rep.m_exact = int(((post["m"].view(np.uint32) == m.view(np.uint32)) & ~tie_s).sum())
+    rep.es_total = rep.m_total = int((~tie_s).sum())
     rel = rel_x(post["x"], x)
     bad = (rel > RTOL) & ~tie_s
     assert not bad.any(), "parameters differ at %d elements (max rel %g)" % (bad.sum(), rel.max())
@@ -167,7 +179,9 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
     ks = list(range(wl.nch)) if chunks is None else list(chunks)
     bounds = {k: (k * wl.C, min(wl.d, (k + 1) * wl.C)) for k in ks}
     stats = {"chunks": ks, "ties_w": 0, "ties_s": 0, "s_exact": 0, "s_total": 0, "S_exact": 0,
-             "S_total": 0, "inexact_chunks": 0, "free_excluded": 0, "free_rel": {}}
+             "S_total": 0, "ew_exact": 0, "ew_total": 0, "es_exact": 0, "es_total": 0,
+             "m_exact": 0, "m_total": 0, "inexact_chunks": 0, "free_excluded": 0,
+             "free_rel": {}}
 
     def grads_of(k):
         lo, hi = bounds[k]
@@ -212,6 +226,7 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
                 post = gpu_chunk_state(opt, x, k, POST)
                 r = check_compressed_step(pre[k], gk[k], post, wl.C, wl.beta1, wl.eps, wl.lr)
                 for f in ("ties_w", "ties_s", "s_exact", "s_total", "S_exact", "S_total",
+                          "ew_exact", "ew_total", "es_exact", "es_total", "m_exact", "m_total",
                           "inexact_chunks"):
                     stats[f] += getattr(r, f)
         if t <= free_steps:
