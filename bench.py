@@ -9,7 +9,11 @@ fp32 parameters, W = 16 simulated workers, C = d/W, bf16 gradients). The metric 
 params x workers / s of the compressed step, with achieved HBM GB/s against the measured copy
 bandwidth. With N > 1 (torchrun, one process per GPU) every rank runs its own replica of the
 whole workload (the method's W workers are simulated inside each GPU; there is no data-path
-collective) and the value is the sum over ranks, timed as the max over ranks.
+collective) and the value is the sum over ranks, timed as the max over ranks. After that
+headline, the same workload runs as N data-parallel ranks (one per GPU, W / N workers each,
+the compressed allreduce between the GPUs fused into the kernels over peer memory), reported in
+the line's "dp" object: its step time (max over ranks), its speed-up over the single-GPU step,
+the bytes each rank stores into its peers per step and every rank's status word.
 
 ``--impl reference`` times the CPU oracle (plain single-threaded C) on a bounded sample of the
 same workload; rank 0 alone runs it.
@@ -55,6 +59,9 @@ def parse_args():
     p.add_argument("--dp", type=int, default=0,
                    help="data-parallel ranks: with one process, R ranks emulated on this GPU; "
                         "under torchrun, one rank per process (R = world size)")
+    p.add_argument("--no-dp-section", action="store_true",
+                   help="under torchrun with N > 1, skip timing the data-parallel step after "
+                        "the replica headline")
     return p.parse_args()
 
 
@@ -240,6 +247,104 @@ def oracle_sample_rate(wl, state, g, seconds):
     return steps * n * wl.W / el, steps, n
 
 
+def dp_ranks_supported(wl, world):
+    """Whether the workload's W workers split evenly over `world` data-parallel ranks (at most
+    eight, the library's limit)."""
+    return 1 < world <= 8 and wl.W % world == 0
+
+
+def dp_subobject(wl, R, ms_max, single_ms, flags_per_rank):
+    """The data-parallel part of the multi-GPU JSON line: the step of R ranks (W / R workers
+    each) timed as the max over ranks, its speed-up over the single-GPU step of the same
+    workload, the bytes each rank stores into other ranks' memory per step, and every rank's
+    status word (bit 4 = a barrier wait ran out)."""
+    flags = [int(f) for f in flags_per_rank]
+    return {"ranks": R, "workers_per_rank": wl.W // R, "ms_per_step": ms_max,
+            "strong_scaling_vs_single": (single_ms / ms_max) if ms_max > 0 else None,
+            "nvlink_bytes_per_rank_per_step": wl.dp_nvlink_bytes_per_rank(R),
+            "status_flags_per_rank": flags,
+            "timeout_seen": any(f & 4 for f in flags)}
+
+
+def time_dp_process_ranks(wl, R, rank, dev, steps, warmup, warm_steps=None, sampler=None):
+    """One data-parallel rank per process (this process is `rank` of R, connected to the others
+    through CUDA IPC over the default process group): warm-up, freeze, `warmup` untimed and
+    `steps` timed compressed steps. Returns (max-over-ranks ms for the timed steps, this rank's
+    status word, the warm-up ms per step, rank 0's per-kernel ms per step). Every rank takes the
+    same collective steps in the same order."""
+    import torch
+    import torch.distributed as dist
+
+    from communication_compressed_optimizer_momentum_b200 import dp
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+    Wl = wl.W // R
+    dt = wls.torch_dtype(wl)
+    x = wls.torch_params(wl, dev)
+    g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
+    opt = dp.OneBitAdamRank(wl.d, wl.W, wl.C, R, rank, wl.beta1, wl.beta2, wl.eps,
+                            grad_dtype=dt, device=dev)
+    dp.connect_process_group(opt)
+
+    def mine(phase, t):
+        wls.torch_fill_grads(wl, g, phase, t)
+        v = g[rank * Wl:(rank + 1) * Wl]
+        return v if v.data_ptr() % 16 == 0 else v.clone()
+    warm_ms = []
+    for t in range(wl.warmup_steps if warm_steps is None else warm_steps):
+        gr = mine(0, t)
+        w0 = torch.cuda.Event(enable_timing=True)
+        w1 = torch.cuda.Event(enable_timing=True)
+        w0.record()
+        opt.warmup_step(x, gr, wl.lr)
+        w1.record()
+        w1.synchronize()
+        warm_ms.append(w0.elapsed_time(w1))
+    opt.freeze()
+    gr = mine(1, 1)
+    torch.cuda.synchronize()
+    for _ in range(max(warmup, 0)):
+        opt.step(x, gr, wl.lr)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    opt.timing(steps)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.mark("t0")
+    t0.record(stream)
+    for _ in range(steps):
+        opt.step(x, gr, wl.lr)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.mark("t1")
+    dist.barrier()
+    ms = t0.elapsed_time(t1)
+    kms, nrec = opt.timing_read()
+    opt.timing(0)
+    ms_max = max_over_ranks(ms, dev)
+    flags = opt.status()
+    # every rank's exchange region stays mapped until all ranks are done with it
+    torch.cuda.synchronize()
+    dist.barrier()
+    opt.close()
+    del x, g, gr
+    torch.cuda.empty_cache()
+    return ms_max, flags, warm_ms, {k: v / max(nrec, 1) for k, v in kms.items()}
+
+
+def gather_flags(flags, world):
+    """Every rank's status word, in rank order (the flags themselves with one rank)."""
+    import torch.distributed as dist
+    if world == 1 or not (dist.is_available() and dist.is_initialized()):
+        return [int(flags)]
+    out = [0] * world
+    dist.all_gather_object(out, int(flags))
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -369,6 +474,7 @@ def run_ours(args):
                          "compressed step(s), single-threaded C" % (n, wl.W, n_steps),
                "host": host_cpu()}
 
+    line = None
     if rank == 0:
         from communication_compressed_optimizer_momentum_b200 import workloads as _w
         line = {
@@ -395,8 +501,29 @@ def run_ours(args):
             "gpu_launches": opt.info()["launches_per_step"] * args.steps,
             "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "status_flags": status,
         }
-        print(json.dumps(line), flush=True)
     opt.close()
+    if world > 1:
+        # after the replica headline, the same workload as data-parallel ranks: one rank per
+        # GPU, W / N workers each, the compressed allreduce between the GPUs fused into the
+        # kernels over peer memory (the same collective steps on every rank)
+        del x, g
+        torch.cuda.empty_cache()
+        dp_obj = None
+        if args.no_dp_section:
+            dp_obj = {"skipped": "--no-dp-section"}
+        elif not dp_ranks_supported(wl, world):
+            dp_obj = {"skipped": "the workload's %d workers do not split over %d ranks"
+                                 % (wl.W, world)}
+        else:
+            dms, dflags, _, dkms = time_dp_process_ranks(wl, world, rank, dev, args.steps,
+                                                         args.warmup, warm_steps=3)
+            flags_all = gather_flags(dflags, world)
+            dp_obj = dp_subobject(wl, world, dms / args.steps, ms_max / args.steps, flags_all)
+            dp_obj["rank0_kernel_ms_per_step"] = dkms
+        if line is not None:
+            line["dp"] = dp_obj
+    if line is not None:
+        print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -430,35 +557,24 @@ def run_dp(args):
                          % (R, wl.W, R))
     Wl = wl.W // R
     dt = wls.torch_dtype(wl)
-    x0 = wls.torch_params(wl, dev)
+    sampler = ClockSampler(local)
+    single_ms = None
     if real:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=dev)
-        opt = dp.OneBitAdamRank(wl.d, wl.W, wl.C, R, rank, wl.beta1, wl.beta2, wl.eps,
-                                grad_dtype=dt, device=dev)
-        dp.connect_process_group(opt)
-        handles = [opt]
-        xs = [x0]
-        g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
-
-        def fill(phase, t):
-            wls.torch_fill_grads(wl, g, phase, t)
-            v = g[rank * Wl:(rank + 1) * Wl]
-            return [v if v.data_ptr() % 16 == 0 else v.clone()]
-
-        def warm_step(gs):
-            opt.warmup_step(xs[0], gs[0], wl.lr)
-
-        def step(gs):
-            opt.step(xs[0], gs[0], wl.lr)
-
-        def freeze():
-            opt.freeze()
+        sampler.start()
+        time.sleep(0.5)
+        ms_max, flags, warm_ms, kernel_ms = time_dp_process_ranks(
+            wl, R, rank, dev, args.steps, args.warmup, sampler=sampler)
+        clocks = sampler.stop()
+        status = 0
+        for f in gather_flags(flags, world):
+            status |= f
         launches = 7
     else:
+        x0 = wls.torch_params(wl, dev)
         em = dp.EmulatedRanks(wl.d, wl.W, wl.C, R, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
                               device=dev)
-        handles = em.ranks
         xs = [x0.clone() for _ in range(R)]
         g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
 
@@ -469,75 +585,52 @@ def run_dp(args):
                 v = g[r * Wl:(r + 1) * Wl]
                 out.append(v if v.data_ptr() % 16 == 0 else v.clone())
             return out
-
-        def warm_step(gs):
-            em.warmup_step(xs, gs, wl.lr)
-
-        def step(gs):
-            em.step(xs, gs, wl.lr)
-
-        def freeze():
-            em.freeze()
         launches = 9 * R                  # phase by phase: a signal and a wait launch each
-    warm_ms = []
-    for t in range(wl.warmup_steps):
-        gs = fill(0, t)
-        w0 = torch.cuda.Event(enable_timing=True)
-        w1 = torch.cuda.Event(enable_timing=True)
-        w0.record()
-        warm_step(gs)
-        w1.record()
-        w1.synchronize()
-        warm_ms.append(w0.elapsed_time(w1))
-    freeze()
-    gs = fill(1, 1)
-    torch.cuda.synchronize()
-    for _ in range(max(args.warmup, 0)):
-        step(gs)
-    torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.5)
-    # per-kernel events of rank 0 (only meaningful when its launches are not interleaved with
-    # other emulated ranks': one process per rank, or a single rank)
-    per_kernel = real or R == 1
-    if per_kernel:
-        handles[0].timing(args.steps)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    if real:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t0.record(stream)
-    for _ in range(args.steps):
-        step(gs)
-    t1.record(stream)
-    torch.cuda.synchronize()
-    if real:
-        dist.barrier()
-    ms = t0.elapsed_time(t1)
-    kernel_ms = None
-    if per_kernel:
-        kms, nrec = handles[0].timing_read()
-        handles[0].timing(0)
-        kernel_ms = {k: v / max(nrec, 1) for k, v in kms.items()}
-    time.sleep(0.3)
-    clocks = sampler.stop()
-    ms_max = max_over_ranks(ms, dev)
-    status = 0
-    for h in handles:
-        status |= h.status()
-    peak, peak_src = measured_hbm_peak()
-    n_gpu = max(world, 1)
-    step_bytes = wl.dp_algorithmic_bytes_per_param(R) * wl.d
-    achieved = step_bytes * args.steps / (ms_max / 1e3) / 1e9
-    single_ms = None
-    if world == 1:
+        warm_ms = []
+        for t in range(wl.warmup_steps):
+            gs = fill(0, t)
+            w0 = torch.cuda.Event(enable_timing=True)
+            w1 = torch.cuda.Event(enable_timing=True)
+            w0.record()
+            em.warmup_step(xs, gs, wl.lr)
+            w1.record()
+            w1.synchronize()
+            warm_ms.append(w0.elapsed_time(w1))
+        em.freeze()
+        gs = fill(1, 1)
+        torch.cuda.synchronize()
+        for _ in range(max(args.warmup, 0)):
+            em.step(xs, gs, wl.lr)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        sampler.start()
+        time.sleep(0.5)
+        # per-kernel events of rank 0: only meaningful when its launches are not interleaved
+        # with other emulated ranks' (a single rank)
+        if R == 1:
+            em.ranks[0].timing(args.steps)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        sampler.mark("t0")
+        t0.record(stream)
+        for _ in range(args.steps):
+            em.step(xs, gs, wl.lr)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        sampler.mark("t1")
+        ms_max = t0.elapsed_time(t1)
+        kernel_ms = None
+        if R == 1:
+            kms, nrec = em.ranks[0].timing_read()
+            em.ranks[0].timing(0)
+            kernel_ms = {k: v / max(nrec, 1) for k, v in kms.items()}
+        time.sleep(0.3)
+        clocks = sampler.stop()
+        status = em.status()
         # the single-GPU step of the same workload, same process, for comparison
-        for h in handles:
-            h.close()
-        del handles, xs
+        em.close()
+        del em, xs
         torch.cuda.empty_cache()
         one = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
                             device=dev)
@@ -556,9 +649,10 @@ def run_dp(args):
         torch.cuda.synchronize()
         single_ms = s0.elapsed_time(s1) / args.steps
         one.close()
-    else:
-        for h in handles:
-            h.close()
+    peak, peak_src = measured_hbm_peak()
+    n_gpu = max(world, 1)
+    step_bytes = wl.dp_algorithmic_bytes_per_param(R) * wl.d
+    achieved = step_bytes * args.steps / (ms_max / 1e3) / 1e9
     if rank == 0:
         line = {
             "metric": METRIC, "value": whole_job_rate(wl.d * wl.W * args.steps, 1, ms_max),

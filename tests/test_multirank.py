@@ -72,3 +72,56 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["unit"] == "params*workers/s" and line["higher_is_better"] is True
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def _dp_rank_main(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    import bench
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+    wl = wls.WORKLOADS["bert_large_bucket"]
+    flags = 4 if rank == 1 else 0               # rank 1's barrier wait ran out
+    ms_max = bench.max_over_ranks(8.0 + rank, "cpu")
+    all_flags = bench.gather_flags(flags, world)
+    obj = bench.dp_subobject(wl, world, ms_max, 9.4, all_flags)
+    q.put((rank, obj))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_data_parallel_subobject_gloo():
+    """Under torchrun with N > 1 the benchmark adds a "dp" object: the data-parallel step timed
+    as the max over ranks, its speed-up over the single-GPU step, the bytes a rank stores into
+    its peers per step and every rank's status word, gathered in rank order."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dp_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    d, W = 333_563_904, 16
+    for rank in (0, 1):
+        obj = out[rank]
+        assert obj["ranks"] == 2 and obj["workers_per_rank"] == 8
+        assert obj["ms_per_step"] == 9.0                       # the slower rank's time
+        assert obj["strong_scaling_vs_single"] == pytest.approx(9.4 / 9.0)
+        assert obj["nvlink_bytes_per_rank_per_step"] == pytest.approx((W / 2 + 1) * d / 16)
+        assert obj["status_flags_per_rank"] == [0, 4]
+        assert obj["timeout_seen"] is True
+
+
+def test_data_parallel_section_only_where_workers_split():
+    sys.path.insert(0, ROOT)
+    import bench
+    from communication_compressed_optimizer_momentum_b200 import workloads as wls
+    wl = wls.WORKLOADS["bert_large_bucket"]                    # W = 16
+    assert [n for n in range(1, 10) if bench.dp_ranks_supported(wl, n)] == [2, 4, 8]
+    assert not bench.dp_ranks_supported(wls.sweep_workload(2, None), 4)
