@@ -1,13 +1,16 @@
-"""CPU oracle for the compression phase of 1-bit Adam (arXiv 2102.02888).
+"""CPU oracle for the compression phase of 1-bit Adam (arXiv 2102.02888) and of its 0/1 Adam
+variant.
 
-TEST INFRASTRUCTURE ONLY. This package wraps ``onebit_oracle.c``, a plain single-threaded C
-restatement of the method, with ctypes and numpy. Only the test suite, the package's smoke
-check and the benchmark's CPU-baseline leg (and its ``--impl reference`` arm) may import it; the
-product path (the CUDA library and its binding) never does, and the two share no code.
+TEST INFRASTRUCTURE ONLY. This package wraps ``onebit_oracle.c`` and ``zero_one_oracle.c``,
+plain single-threaded C restatements of the methods, with ctypes and numpy. Only the test suite,
+the package's smoke check and the benchmark's CPU-baseline leg (and its ``--impl reference`` arm)
+may import it; the product path (the CUDA library and its binding) never does, and the two share
+no code.
 
 All arrays are numpy, C-contiguous. Grads are float32 ``[W][d]`` or bf16 bit patterns stored as
-uint16 ``[W][d]``. Every function follows the conventions R1-R11 stated at the top of the C
-file; each cites the page and section it restates.
+uint16 ``[W][d]``. Every function follows the conventions R1-R11 (and, for the ``zo_*``
+functions of the 0/1 Adam variant, Z1-Z7) stated at the top of the C files; each cites the page
+and section it restates.
 """
 from __future__ import annotations
 
@@ -19,6 +22,8 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "onebit_oracle.c")
+_SRC01 = os.path.join(_HERE, "zero_one_oracle.c")
+SOURCES = (_SRC, _SRC01)
 _LIB = os.path.join(_HERE, "libonebit_oracle.so")
 
 # Flags that keep every fp32 operation a single IEEE operation (R7): no contraction to FMA, no
@@ -29,9 +34,10 @@ CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-s
 
 def build(force: bool = False) -> str:
     """Compile the oracle to ``oracle/libonebit_oracle.so`` (gcc) if missing or stale."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    if force or not os.path.exists(_LIB) or any(
+            os.path.getmtime(_LIB) < os.path.getmtime(src) for src in SOURCES):
         tmp = _LIB + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, *SOURCES, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -65,6 +71,17 @@ def _load(path: str):
     L.oracle_compressed_step.argtypes = [i64, i32, i64, f32, f32, f32, P, P, P, P, P, P,
                                          c_int, P, P, P, P, P]
     L.oracle_compressed_step.restype = i64
+    L.oracle01_local.argtypes = [i64, i32, f32, f32, P, P, P, c_int]
+    L.oracle01_local.restype = None
+    L.oracle01_compress.argtypes = [i64, i32, i64, P, P, P, P]
+    L.oracle01_compress.restype = None
+    L.oracle01_apply.argtypes = [i64, i64, f32, f32, f32, c_int, P, P, P, P, P]
+    L.oracle01_apply.restype = None
+    L.oracle01_step.argtypes = [i64, i32, i64, f32, f32, f32, f32, f32, c_int, c_int, P, P, P,
+                                P, P, P, P, c_int, P, P, P, P, P, P]
+    L.oracle01_step.restype = i64
+    L.oracle01_local_model.argtypes = [i64, f32, P, P, P, P]
+    L.oracle01_local_model.restype = None
     return L
 
 
@@ -218,6 +235,135 @@ class OracleState:
         assert self.frozen
         return compressed_step(self.x, self.m, self.v, self.e_w, self.e_s, g, self.C,
                                self.beta1, self.eps, lr)
+
+
+# ----------------------------------------------------------------------------------------------
+# the 0/1 Adam variant (zero_one_oracle.c, readings Z1-Z7)
+
+def _wd(a, W, d, name):
+    assert a.dtype == np.float32 and a.shape == (W, d) and a.flags["C_CONTIGUOUS"], name
+
+
+def zo_local(m_w, u_w, g, beta1, lr):
+    """Z3: every worker's local step, in place on m_w and u_w ([W][d])."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    _wd(m_w, W, d, "m_w")
+    _wd(u_w, W, d, "u_w")
+    lib().oracle01_local(d, W, beta1, lr, _p(m_w), _p(u_w), _p(g), gt)
+
+
+def zo_compress(u_w, e_w, C):
+    """Z4, worker side: 1-bit messages of the accumulated updates; e_w updated in place.
+
+    Returns (s [W][nch] float32, bits_w [W][ceil(d/32)] uint32)."""
+    u_w = _f32(u_w)
+    W, d = u_w.shape
+    _wd(e_w, W, d, "e_w")
+    s = np.zeros((W, nchunks(d, C)), dtype=np.float32)
+    bits = np.zeros((W, nwords(d)), dtype=np.uint32)
+    lib().oracle01_compress(d, W, C, _p(u_w), _p(e_w), _p(s), _p(bits))
+    return s, bits
+
+
+def zo_apply(bits_s, S, v, x, C, eps, gamma, beta2, refresh):
+    """Z5-Z6: the synchronised step from the server message, in place on x (and on v when
+    `refresh`). Returns mbar [d]."""
+    d = x.size
+    bits_s = np.ascontiguousarray(bits_s, dtype=np.uint32)
+    S = _f32(S)
+    for a in (v, x):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    mbar = np.zeros(d, dtype=np.float32)
+    lib().oracle01_apply(d, C, eps, gamma, beta2, 1 if refresh else 0, _p(bits_s), _p(S),
+                         _p(v), _p(x), _p(mbar))
+    return mbar
+
+
+def zo_step(x, m_w, u_w, v, e_w, e_s, g, C, beta1, beta2, eps, lr, gamma, sync, refresh):
+    """One step of the variant's compression phase (Z3, and Z4-Z6 when `sync`), in place on
+    x, m_w, u_w, v, e_w, e_s. Returns the synchronisation's messages (s, S, bits_w, bits_s,
+    mbar, inexact), or None without one."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    for a, nm in ((m_w, "m_w"), (u_w, "u_w"), (e_w, "e_w")):
+        _wd(a, W, d, nm)
+    for a in (x, v, e_s):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    nch = nchunks(d, C)
+    s = np.zeros((W, nch), dtype=np.float32)
+    S = np.zeros(nch, dtype=np.float32)
+    bits_w = np.zeros((W, nwords(d)), dtype=np.uint32)
+    bits_s = np.zeros(nwords(d), dtype=np.uint32)
+    mbar = np.zeros(d, dtype=np.float32)
+    z = np.zeros(d, dtype=np.float32)
+    inexact = lib().oracle01_step(d, W, C, beta1, beta2, eps, lr, gamma, 1 if sync else 0,
+                                  1 if refresh else 0, _p(x), _p(m_w), _p(u_w), _p(v), _p(e_w),
+                                  _p(e_s), _p(g), gt, _p(s), _p(S), _p(bits_w), _p(bits_s),
+                                  _p(mbar), _p(z))
+    if not sync:
+        return None
+    return {"s": s, "S": S, "bits_w": bits_w, "bits_s": bits_s, "mbar": mbar,
+            "inexact": int(inexact)}
+
+
+def zo_local_model(x, u, v, eps):
+    """Z7: a worker's local model x - u / (sqrt(v) + eps)."""
+    x, u, v = _f32(x), _f32(u), _f32(v)
+    out = np.zeros(x.size, dtype=np.float32)
+    lib().oracle01_local_model(x.size, eps, _p(x), _p(u), _p(v), _p(out))
+    return out
+
+
+class ZeroOneState:
+    """The 0/1 Adam variant's state on the host: x, m, v through the warm-up (shared with
+    1-bit Adam, Z1); after the freeze every worker's momentum and accumulated update, the
+    explicit residuals, and the schedule: a synchronisation every H steps, a variance refresh
+    at every K-th synchronisation (K = 0: never), Gamma the fp32 sum of the learning rates since
+    the last synchronisation (Z2-Z6)."""
+
+    def __init__(self, x, W, C, H, K, beta1=0.9, beta2=0.999, eps=1e-8):
+        assert H >= 1 and K >= 0
+        self.x = _f32(x).copy()
+        d = self.x.size
+        self.d, self.W, self.C, self.H, self.K = d, W, C, H, K
+        self.beta1, self.beta2, self.eps = beta1, beta2, eps
+        self.m = np.zeros(d, dtype=np.float32)
+        self.v = np.zeros(d, dtype=np.float32)
+        self.frozen = False
+        self.t = 0
+        self.syncs = 0
+        self.gamma = np.float32(0.0)
+
+    def warmup_step(self, g, lr):
+        assert not self.frozen
+        warmup_step(self.x, self.m, self.v, g, self.beta1, self.beta2, self.eps, lr)
+
+    def freeze(self):
+        """Z2: every worker starts from the warm-up momentum, with u_w = e_w = e_s = 0."""
+        self.frozen = True
+        self.m_w = np.ascontiguousarray(np.broadcast_to(self.m, (self.W, self.d)),
+                                        dtype=np.float32)
+        self.u_w = np.zeros((self.W, self.d), dtype=np.float32)
+        self.e_w = np.zeros((self.W, self.d), dtype=np.float32)
+        self.e_s = np.zeros(self.d, dtype=np.float32)
+
+    def step(self, g, lr):
+        assert self.frozen
+        self.t += 1
+        self.gamma = np.float32(self.gamma + np.float32(lr))
+        sync = self.t % self.H == 0
+        refresh = sync and self.K > 0 and (self.syncs + 1) % self.K == 0
+        out = zo_step(self.x, self.m_w, self.u_w, self.v, self.e_w, self.e_s, g, self.C,
+                      self.beta1, self.beta2, self.eps, lr, float(self.gamma), sync, refresh)
+        if sync:
+            self.syncs += 1
+            self.gamma = np.float32(0.0)
+            out["refresh"] = refresh
+        return out
+
+    def local_model(self, w):
+        return zo_local_model(self.x, self.u_w[w], self.v, self.eps)
 
 
 class use_library:

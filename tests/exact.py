@@ -132,3 +132,80 @@ def exact_compressed_step(x, m, v, e_w, e_s, g, C, beta1, eps, lr):
         new_x[i] = r32(fr(x[i]) - fr(upd))
     return {"xw": xw, "s": s, "bits_w": bits, "e_w": new_ew, "y": y, "z": z, "S": S,
             "bits_s": z >= 0, "e_s": new_es, "m": new_m, "x": new_x}
+
+
+def exact_zero_one_run(x, m, v, g_list, lr_list, C, H, K, beta1, beta2, eps):
+    """Exact re-derivation of the 0/1 Adam variant's compression phase (tiny inputs only): from
+    the state at the freeze (x, shared m, v; residuals zero) through the steps of g_list
+    ([W][d] float32 each) with learning rates lr_list; a synchronisation after every H-th step,
+    a variance refresh at every K-th synchronisation (K = 0: never). Every fp32 operation is the
+    exact rational result rounded once to binary32 and norms are summed exactly.
+
+    Returns the final x, v, m_w, u_w, e_w, e_s and the list of each synchronisation's
+    messages (s, bits_w, S, bits_s, mbar)."""
+    g0 = np.asarray(g_list[0], dtype=np.float32)
+    W, d = g0.shape
+    nch = (d + C - 1) // C
+    b1, b2 = fr(beta1), fr(beta2)
+    omb1, omb2 = fr(r32(1 - b1)), fr(r32(1 - b2))
+    x = np.array(x, dtype=np.float32)
+    v = np.array(v, dtype=np.float32)
+    m_w = np.array(np.broadcast_to(np.asarray(m, dtype=np.float32), (W, d)), dtype=np.float32)
+    u_w = np.zeros((W, d), dtype=np.float32)
+    e_w = np.zeros((W, d), dtype=np.float32)
+    e_s = np.zeros(d, dtype=np.float32)
+    gamma = np.float32(0.0)
+    syncs = []
+    for t, (g, lr) in enumerate(zip(g_list, lr_list), start=1):
+        g = np.asarray(g, dtype=np.float32)
+        lrf = fr(lr)
+        for w in range(W):
+            for i in range(d):
+                m_w[w, i] = r32(fr(r32(b1 * fr(m_w[w, i]))) + fr(r32(omb1 * fr(g[w, i]))))
+                u_w[w, i] = r32(fr(u_w[w, i]) + fr(r32(lrf * fr(m_w[w, i]))))
+        gamma = r32(fr(gamma) + lrf)
+        if t % H:
+            continue
+        xw = np.zeros((W, d), dtype=np.float32)
+        for w in range(W):
+            for i in range(d):
+                xw[w, i] = r32(fr(u_w[w, i]) + fr(e_w[w, i]))
+        bits = xw >= 0
+        s = np.zeros((W, nch), dtype=np.float32)
+        for w in range(W):
+            for k in range(nch):
+                lo, hi = k * C, min(d, (k + 1) * C)
+                ss = sum((fr(xw[w, i]) ** 2 for i in range(lo, hi)), F(0))
+                s[w, k] = r32_sqrt(ss / (hi - lo))
+                for i in range(lo, hi):
+                    q = fr(s[w, k]) if bits[w, i] else -fr(s[w, k])
+                    e_w[w, i] = r32(fr(xw[w, i]) - q)
+        z = np.zeros(d, dtype=np.float32)
+        S = np.zeros(nch, dtype=np.float32)
+        for k in range(nch):
+            lo, hi = k * C, min(d, (k + 1) * C)
+            for i in range(lo, hi):
+                acc = sum(((fr(s[w, k]) if bits[w, i] else -fr(s[w, k])) for w in range(W)),
+                          F(0))
+                y = r32(acc / W)
+                z[i] = r32(fr(y) + fr(e_s[i]))
+            ss = sum((fr(z[i]) ** 2 for i in range(lo, hi)), F(0))
+            S[k] = r32_sqrt(ss / (hi - lo))
+            for i in range(lo, hi):
+                e_s[i] = r32(fr(z[i]) - (fr(S[k]) if z[i] >= 0 else -fr(S[k])))
+        refresh = K > 0 and (len(syncs) + 1) % K == 0
+        mbar = np.zeros(d, dtype=np.float32)
+        for i in range(d):
+            k = i // C
+            ubar = fr(S[k]) if z[i] >= 0 else -fr(S[k])
+            den = r32(fr(r32_sqrt(fr(v[i]))) + fr(eps))
+            x[i] = r32(fr(x[i]) - fr(r32(ubar / fr(den))))
+            mbar[i] = r32(ubar / fr(gamma))
+            if refresh:
+                v[i] = r32(fr(r32(b2 * fr(v[i]))) + fr(r32(omb2 * fr(r32(fr(mbar[i]) ** 2)))))
+        m_w[:] = mbar
+        u_w[:] = 0.0
+        gamma = np.float32(0.0)
+        syncs.append({"s": s, "bits_w": bits, "S": S, "bits_s": z >= 0, "mbar": mbar,
+                      "refresh": refresh})
+    return {"x": x, "v": v, "m_w": m_w, "u_w": u_w, "e_w": e_w, "e_s": e_s, "syncs": syncs}
