@@ -23,7 +23,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "onebit_oracle.c")
 _SRC01 = os.path.join(_HERE, "zero_one_oracle.c")
-SOURCES = (_SRC, _SRC01)
+_SRCBC = os.path.join(_HERE, "bias_corrected_oracle.c")
+SOURCES = (_SRC, _SRC01, _SRCBC)
 _LIB = os.path.join(_HERE, "libonebit_oracle.so")
 
 # Flags that keep every fp32 operation a single IEEE operation (R7): no contraction to FMA, no
@@ -82,6 +83,10 @@ def _load(path: str):
     L.oracle01_step.restype = i64
     L.oracle01_local_model.argtypes = [i64, f32, P, P, P, P]
     L.oracle01_local_model.restype = None
+    L.oracle_warmup_step_bc.argtypes = [i64, i32, f32, f32, f32, f32, f32, f32, P, P, P, P, c_int]
+    L.oracle_warmup_step_bc.restype = None
+    L.oracle_freeze_bc.argtypes = [i64, f32, f32, P, P]
+    L.oracle_freeze_bc.restype = None
     return L
 
 
@@ -139,6 +144,38 @@ def warmup_step(x, m, v, g, beta1, beta2, eps, lr):
     for a in (x, m, v):
         assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
     lib().oracle_warmup_step(d, W, beta1, beta2, eps, lr, _p(x), _p(m), _p(v), _p(g), gt)
+
+
+def bias_corrections(beta1, beta2, t):
+    """(c1_t, c2_t) = (1 - beta1^t, 1 - beta2^t): beta^t the fp64 product of t factors beta (the
+    fp32 value) in order, 1 - beta^t in fp64, rounded once to fp32 (reading B1 of
+    bias_corrected_oracle.c; fp32 arithmetic would lose most digits of 1 - beta2^t to
+    cancellation)."""
+    p1 = p2 = 1.0
+    b1, b2 = float(np.float32(beta1)), float(np.float32(beta2))
+    for _ in range(t):
+        p1 *= b1
+        p2 *= b2
+    return float(np.float32(1.0 - p1)), float(np.float32(1.0 - p2))
+
+
+def warmup_step_bc(x, m, v, g, beta1, beta2, eps, lr, t):
+    """Bias-corrected warm-up step t (1-based), in place on x, m, v (m and v stay
+    uncorrected; reading B1)."""
+    g, gt = _grads(g)
+    W, d = g.shape
+    for a in (x, m, v):
+        assert a.dtype == np.float32 and a.shape == (d,) and a.flags["C_CONTIGUOUS"]
+    c1, c2 = bias_corrections(beta1, beta2, t)
+    lib().oracle_warmup_step_bc(d, W, beta1, beta2, eps, lr, c1, c2, _p(x), _p(m), _p(v),
+                                _p(g), gt)
+
+
+def freeze_bc(m, v, beta1, beta2, T):
+    """The freeze after T bias-corrected warm-up steps: m = m / c1_T, v = v / c2_T (B1)."""
+    assert m.dtype == np.float32 and v.dtype == np.float32 and m.shape == v.shape
+    c1, c2 = bias_corrections(beta1, beta2, T)
+    lib().oracle_freeze_bc(m.size, c1, c2, _p(m), _p(v))
 
 
 def worker(m, g, e_w, C, beta1):
@@ -210,11 +247,13 @@ class OracleState:
     explicit worker and server residuals. Mirrors the phases of the method: warm-up steps, the
     variance freeze, compressed steps."""
 
-    def __init__(self, x, W, C, beta1=0.9, beta2=0.999, eps=1e-8):
+    def __init__(self, x, W, C, beta1=0.9, beta2=0.999, eps=1e-8, bias_correction=False):
         self.x = _f32(x).copy()
         d = self.x.size
         self.d, self.W, self.C = d, W, C
         self.beta1, self.beta2, self.eps = beta1, beta2, eps
+        self.bias_correction = bias_correction
+        self.t = 0
         self.m = np.zeros(d, dtype=np.float32)
         self.v = np.zeros(d, dtype=np.float32)
         self.e_w = None
@@ -223,10 +262,18 @@ class OracleState:
 
     def warmup_step(self, g, lr):
         assert not self.frozen
-        warmup_step(self.x, self.m, self.v, g, self.beta1, self.beta2, self.eps, lr)
+        self.t += 1
+        if self.bias_correction:
+            warmup_step_bc(self.x, self.m, self.v, g, self.beta1, self.beta2, self.eps, lr,
+                           self.t)
+        else:
+            warmup_step(self.x, self.m, self.v, g, self.beta1, self.beta2, self.eps, lr)
 
     def freeze(self):
-        """Freeze v as the preconditioner; residuals start at zero (R11)."""
+        """Freeze v as the preconditioner; residuals start at zero (R11). After a
+        bias-corrected warm-up, m and v continue corrected (B1)."""
+        if self.bias_correction and self.t > 0:
+            freeze_bc(self.m, self.v, self.beta1, self.beta2, self.t)
         self.frozen = True
         self.e_w = np.zeros((self.W, self.d), dtype=np.float32)
         self.e_s = np.zeros(self.d, dtype=np.float32)

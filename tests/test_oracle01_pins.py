@@ -1,6 +1,6 @@
 """The 0/1 Adam variant's oracle against its pins, and planted mistakes that the pins must
 catch (each mutant is a copy of zero_one_oracle.c with one plausible error, built with the
-unchanged 1-bit Adam oracle; the mistakes are planted on the CPU only)."""
+oracle's other, unchanged files; the mistakes are planted on the CPU only)."""
 import os
 import subprocess
 
@@ -10,7 +10,6 @@ import oracle
 from oracle01_pins import PINS01
 
 SRC01 = os.path.join(os.path.dirname(oracle.__file__), "zero_one_oracle.c")
-SRC = os.path.join(os.path.dirname(oracle.__file__), "onebit_oracle.c")
 
 MUTANTS01 = {
     "accumulate_drops_lr": ("float step = lr * m_w[j];", "float step = m_w[j];"),
@@ -48,7 +47,8 @@ def test_pins_catch_planted_mistake(name, src01_text, tmp_path):
     c = tmp_path / "mutant01.c"
     c.write_text(src01_text.replace(old, new))
     so = tmp_path / "mutant01.so"
-    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), SRC, str(c), "-lm"])
+    others = [src for src in oracle.SOURCES if src != SRC01]
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), *others, str(c), "-lm"])
     caught = []
     with oracle.use_library(str(so)):
         for pin in PINS01:

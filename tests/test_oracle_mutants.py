@@ -11,7 +11,6 @@ import oracle
 from oracle_pins import PINS
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "onebit_oracle.c")
-SRC01 = os.path.join(os.path.dirname(oracle.__file__), "zero_one_oracle.c")
 
 MUTANTS = {
     "worker_drops_residual": ("e[i] = mw + e[i];", "e[i] = mw;"),
@@ -62,8 +61,9 @@ def test_pins_catch_planted_mistake(name, src_text, tmp_path):
     c = tmp_path / "mutant.c"
     c.write_text(mutated)
     so = tmp_path / "mutant.so"
-    # the mutant is linked with the unchanged 0/1 Adam oracle, which the library also holds
-    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), str(c), SRC01, "-lm"])
+    # the mutant is linked with the oracle's other files, unchanged
+    others = [src for src in oracle.SOURCES if src != SRC]
+    subprocess.check_call(["gcc", *oracle.CFLAGS, "-o", str(so), str(c), *others, "-lm"])
     caught = []
     with oracle.use_library(str(so)):
         for pin in PINS:
