@@ -32,7 +32,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "step_kernels_bert_large_bucket.md")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "dram_traffic_bert_large_bucket.json")
 KERNEL_SRC = os.path.join(ROOT, "communication_compressed_optimizer_momentum_b200", "csrc",
                           "kernels.cuh")
 FALLBACK_HBM_GBS = 6650.0
@@ -59,6 +59,12 @@ def parse_args():
     p.add_argument("--dp", type=int, default=0,
                    help="data-parallel ranks: with one process, R ranks emulated on this GPU; "
                         "under torchrun, one rank per process (R = world size)")
+    p.add_argument("--variant", default="onebit", choices=("onebit", "zero_one"),
+                   help="zero_one: the 0/1 Adam variant's compression phase (local steps and a "
+                        "synchronisation every --sync-every steps)")
+    p.add_argument("--sync-every", type=int, default=4, help="0/1 Adam: H")
+    p.add_argument("--refresh-every", type=int, default=2,
+                   help="0/1 Adam: variance refresh every K-th synchronisation (0: never)")
     p.add_argument("--no-dp-section", action="store_true",
                    help="under torchrun with N > 1, skip timing the data-parallel step after "
                         "the replica headline")
@@ -93,26 +99,23 @@ def kernel_source_sha():
 
 
 def ncu_traffic(workload):
-    """DRAM bytes per worker-kernel launch from the committed ncu summary, if it was taken on
-    the current kernel source for this workload; otherwise None."""
+    """DRAM bytes per launch of the step's kernels at the workload's full size, from the
+    committed ncu summary (profiles/dram_traffic_bert_large_bucket.json), when it was taken on
+    the current kernel source for this workload: {kernel: bytes}; otherwise {}."""
     try:
-        with open(PROFILE_SUMMARY) as f:
-            text = f.read()
-    except OSError:
-        return None
-    fields = {}
-    for line in text.splitlines():
-        if ":" in line and line.strip().startswith("- "):
-            k, v = line.strip()[2:].split(":", 1)
-            fields[k.strip()] = v.strip().strip("`")
-    if fields.get("kernel_source_sha256") != kernel_source_sha():
-        return None
-    if fields.get("workload") != workload:
-        return None
-    try:
-        return float(fields["dram_bytes_per_launch_full"])
-    except (KeyError, ValueError):
-        return None
+        with open(TRAFFIC_JSON) as f:
+            j = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    if j.get("kernel_source_sha256") != kernel_source_sha() or j.get("workload") != workload:
+        return {}
+    out = {}
+    for name, k in j.get("kernels", {}).items():
+        try:
+            out[name] = float(k["dram_bytes_per_launch_full"])
+        except (KeyError, TypeError, ValueError):
+            continue
+    return out
 
 
 class ClockSampler:
@@ -366,7 +369,15 @@ def run_ours(args):
 
     x = wls.torch_params(wl, dev)
     g = torch.empty((wl.W, wl.d), dtype=dt, device=dev)
-    opt = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt, device=dev)
+    zero_one = args.variant == "zero_one"
+    if zero_one and args.graph:
+        raise SystemExit("--graph: the 0/1 variant's steps differ from step to step")
+    if zero_one:
+        opt = ob.ZeroOneAdam(wl.d, wl.W, wl.C, args.sync_every, args.refresh_every, wl.beta1,
+                             wl.beta2, wl.eps, grad_dtype=dt, device=dev)
+    else:
+        opt = ob.OneBitAdam(wl.d, wl.W, wl.C, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
+                            device=dev)
     warm_ms = []
     for t in range(wl.warmup_steps):             # full-precision Adam warm-up (setup)
         wls.torch_fill_grads(wl, g, 0, t)
@@ -424,10 +435,12 @@ def run_ours(args):
     status = opt.status()
 
     value = whole_job_rate(wl.d * wl.W * args.steps, world, ms_max)
-    step_bytes = wl.algorithmic_bytes_per_param() * wl.d
+    step_bytes = (wl.zero_one_bytes_per_param(args.sync_every, args.refresh_every) if zero_one
+                  else wl.algorithmic_bytes_per_param()) * wl.d
     achieved_step_gbs = step_bytes * args.steps / (ms_max / 1e3) / 1e9
     peak, peak_src = measured_hbm_peak()
     kb = wl.kernel_bytes_per_param()
+    traffic = ncu_traffic(wl.name)
     worker_bytes = kb["worker"] * wl.d
     worker_ms = kernel_ms["worker"] / max(nrec, 1)
     worker_gbs = worker_bytes / (worker_ms / 1e3) / 1e9 if worker_ms > 0 else None
@@ -436,7 +449,7 @@ def run_ours(args):
 
     # end to end through the host-buffer entry point: H2D grads, the step, D2H x
     e2e = None
-    if not args.no_e2e and args.e2e_steps > 0:
+    if not args.no_e2e and args.e2e_steps > 0 and not zero_one:
         g_host = torch.empty((wl.W, wl.d), dtype=dt, pin_memory=True)
         g_host.copy_(g)
         x_host = torch.empty(wl.d, dtype=torch.float32, pin_memory=True)
@@ -460,7 +473,7 @@ def run_ours(args):
         del g_host, x_host
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not zero_one:
         k = 0
         lo, hi = 0, min(wl.d, wl.C)
         st = {"x": _to_np(x[lo:hi]), "m": _to_np(opt.get_chunk_state("m", k)),
@@ -495,12 +508,28 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "kernel": "worker", "achieved": worker_gbs,
                          "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": (worker_gbs / peak) if worker_gbs else None,
-                         "traffic": ncu_traffic(wl.name),
+                         "traffic": traffic.get("worker"),
                          "algorithmic_bytes_per_launch": worker_bytes},
+            # every streaming kernel's ncu DRAM bytes per launch against its algorithmic bytes
+            "traffic_by_kernel": {k2: {"dram_bytes": traffic[k2],
+                                       "algorithmic_bytes": kb[k2] * wl.d,
+                                       "ratio": traffic[k2] / (kb[k2] * wl.d)}
+                                  for k2 in ("worker", "server", "apply") if k2 in traffic},
             "warmup_phase": warmup_phase(wl, warm_ms),
             "gpu_launches": opt.info()["launches_per_step"] * args.steps,
             "clocks": clocks, "e2e": e2e, "cpu_baseline": cpu, "status_flags": status,
         }
+    if line is not None and zero_one:
+        # the variant's steps differ (local ones, a synchronising one every H): the roofline is
+        # the whole step's average bytes against its average time
+        line["config"].update(variant="0/1 Adam", sync_every=args.sync_every,
+                              refresh_every=args.refresh_every)
+        line["roofline"] = {"bound": "hbm", "kernel": "whole step (average over an interval)",
+                            "achieved": achieved_step_gbs, "peak": peak,
+                            "peak_source": peak_src, "unit": "GB/s",
+                            "frac": achieved_step_gbs / peak, "traffic": None,
+                            "algorithmic_bytes_per_launch": step_bytes}
+        line["gpu_launches"] = args.steps + 4 * (args.steps // args.sync_every)
     opt.close()
     if world > 1:
         # after the replica headline, the same workload as data-parallel ranks: one rank per
@@ -511,6 +540,8 @@ def run_ours(args):
         dp_obj = None
         if args.no_dp_section:
             dp_obj = {"skipped": "--no-dp-section"}
+        elif zero_one:
+            dp_obj = {"skipped": "the 0/1 Adam variant runs on one GPU only"}
         elif not dp_ranks_supported(wl, world):
             dp_obj = {"skipped": "the workload's %d workers do not split over %d ranks"
                                  % (wl.W, world)}

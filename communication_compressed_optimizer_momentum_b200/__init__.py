@@ -93,6 +93,11 @@ def onebit_adam_warmup_step(h, x, grads, lr: float, stream=None) -> None:
                                               _stream(stream)), "onebit_adam_warmup_step")
 
 
+def onebit_adam_set_bias_correction(h, on: bool) -> None:
+    _check(_abi.lib().onebit_adam_set_bias_correction(_handle(h), 1 if on else 0),
+           "onebit_adam_set_bias_correction")
+
+
 def onebit_adam_freeze_variance(h, stream=None) -> None:
     _check(_abi.lib().onebit_adam_freeze_variance(_handle(h), _stream(stream)),
            "onebit_adam_freeze_variance")
@@ -231,6 +236,36 @@ def onebit_dp_compressed_phase(h, phase: int, x, grads, lr: float, stream=None) 
                                                  _stream(stream)), "onebit_dp_compressed_phase")
 
 
+def onebit01_init(d: int, W: int, C: int, beta1: float, beta2: float, eps: float, H: int,
+                  K: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_abi.lib().onebit01_init(ctypes.byref(h), d, W, C, beta1, beta2, eps, H, K),
+           "onebit01_init")
+    return h
+
+
+def onebit01_step(h, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit01_step(_handle(h), _ptr(x), _ptr(grads), lr, _stream(stream)),
+           "onebit01_step")
+
+
+def onebit01_info(h) -> dict:
+    out = (ctypes.c_int64 * 6)()
+    _check(_abi.lib().onebit01_info(_handle(h), out), "onebit01_info")
+    keys = ("H", "K", "steps_since_sync", "syncs", "momentum_source", "launches_next_step")
+    return dict(zip(keys, list(out)))
+
+
+def onebit01_get_worker_state(h, which: int, k: int, dst, stream=None) -> None:
+    _check(_abi.lib().onebit01_get_worker_state(_handle(h), which, k, _ptr(dst),
+                                                _stream(stream)), "onebit01_get_worker_state")
+
+
+def onebit01_local_model(h, w: int, x, out, stream=None) -> None:
+    _check(_abi.lib().onebit01_local_model(_handle(h), w, _ptr(x), _ptr(out), _stream(stream)),
+           "onebit01_local_model")
+
+
 def onebit_strerror(code: int) -> str:
     return _abi.lib().onebit_strerror(code).decode()
 
@@ -338,9 +373,12 @@ class OneBitAdam:
     ``freeze()`` (the variance becomes the fixed preconditioner), then ``step`` (compressed)."""
 
     def __init__(self, d: int, W: int, C: int, beta1: float = 0.9, beta2: float = 0.999,
-                 eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None):
-        self._setup(onebit_adam_init(d, W, C, beta1, beta2, eps), d, W, C, grad_dtype, device,
-                    stream)
+                 eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None,
+                 bias_correction: bool = False):
+        h = onebit_adam_init(d, W, C, beta1, beta2, eps)
+        if bias_correction:
+            onebit_adam_set_bias_correction(h, True)
+        self._setup(h, d, W, C, grad_dtype, device, stream)
 
     def _setup(self, h, d, W, C, grad_dtype, device, stream):
         import torch
@@ -424,3 +462,40 @@ class OneBitAdam:
             self.close()
         except Exception:
             pass
+
+
+class ZeroOneAdam(OneBitAdam):
+    """One optimizer instance of the 0/1 Adam variant: the warm-up and the freeze of 1-bit Adam,
+    then ``step`` runs the variant's compression phase -- a local step on every worker, and
+    every H-th step a synchronisation through the compressed allreduce of the workers'
+    accumulated updates, with a variance refresh at every K-th synchronisation (K = 0: never)."""
+
+    WORKER_STATE = {"m_w": 0, "u_w": 1}
+
+    def __init__(self, d: int, W: int, C: int, H: int, K: int, beta1: float = 0.9,
+                 beta2: float = 0.999, eps: float = 1e-8, grad_dtype=None, device="cuda",
+                 stream=None):
+        self.H, self.K = H, K
+        self._setup(onebit01_init(d, W, C, beta1, beta2, eps, H, K), d, W, C, grad_dtype,
+                    device, stream)
+
+    def step(self, x, grads, lr: float, stream=None) -> None:
+        onebit01_step(self.h, x, grads, lr, stream)
+
+    def zo_info(self) -> dict:
+        return onebit01_info(self.h)
+
+    def get_worker_state(self, which: str, k: int = -1, stream=None):
+        """Every worker's momentum ("m_w") or accumulated update ("u_w"): [W][d], or [W][C_k]
+        for chunk k."""
+        import torch
+        n = self.d if k < 0 else min(self.C, self.d - k * self.C)
+        out = torch.empty((self.W, n), dtype=torch.float32, device=self.workspace.device)
+        onebit01_get_worker_state(self.h, self.WORKER_STATE[which], k, out, stream)
+        return out
+
+    def local_model(self, w: int, x, stream=None):
+        import torch
+        out = torch.empty(self.d, dtype=torch.float32, device=self.workspace.device)
+        onebit01_local_model(self.h, w, x, out, stream)
+        return out

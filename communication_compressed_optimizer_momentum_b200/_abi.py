@@ -24,6 +24,7 @@ SIGNATURES = {
     "onebit_adam_bind": (INT, [P, P, ctypes.c_uint64, I32, P]),
     "onebit_adam_warmup_step": (INT, [P, P, P, F32, P]),
     "onebit_adam_freeze_variance": (INT, [P, P]),
+    "onebit_adam_set_bias_correction": (INT, [P, I32]),
     "onebit_adam_compressed_step": (INT, [P, P, P, F32, P]),
     "onebit_adam_compressed_step_host": (INT, [P, P, P, P, P, F32, P]),
     "onebit_adam_host_wait": (INT, [P, P]),
@@ -51,6 +52,11 @@ SIGNATURES = {
     "onebit_dp_set_timeout": (INT, [P, ctypes.c_uint64]),
     "onebit_dp_warmup_phase": (INT, [P, I32, P, P, F32, P]),
     "onebit_dp_compressed_phase": (INT, [P, I32, P, P, F32, P]),
+    "onebit01_init": (INT, [ctypes.POINTER(P), I64, I32, I64, F32, F32, F32, I32, I32]),
+    "onebit01_step": (INT, [P, P, P, F32, P]),
+    "onebit01_info": (INT, [P, ctypes.POINTER(I64)]),
+    "onebit01_get_worker_state": (INT, [P, I32, I64, P, P]),
+    "onebit01_local_model": (INT, [P, I32, P, P, P]),
     "onebit_strerror": (ctypes.c_char_p, [I32]),
     "onebit_last_error": (ctypes.c_char_p, []),
 }

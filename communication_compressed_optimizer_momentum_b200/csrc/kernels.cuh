@@ -148,6 +148,31 @@ __device__ __forceinline__ uint32_t gather_word(uint32_t nib, int lane) {
     return w;
 }
 
+// byte i bit c  ->  byte c bit i, on (lo = bytes 0..3, hi = bytes 4..7): three delta swaps of
+// the row/column index bits; the first two stay inside each 32-bit half.
+__device__ __forceinline__ void transpose8x8(uint32_t& lo, uint32_t& hi) {
+    uint32_t t;
+    t = ((lo >> 7) ^ lo) & 0x00AA00AAu;  lo ^= t ^ (t << 7);
+    t = ((hi >> 7) ^ hi) & 0x00AA00AAu;  hi ^= t ^ (t << 7);
+    t = ((lo >> 14) ^ lo) & 0x0000CCCCu; lo ^= t ^ (t << 14);
+    t = ((hi >> 14) ^ hi) & 0x0000CCCCu; hi ^= t ^ (t << 14);
+    t = ((hi << 4) ^ lo) & 0xF0F0F0F0u;  lo ^= t;  hi ^= t >> 4;
+}
+
+// Byte `b` (0..3) of 8 words -> lo/hi whose byte i is word i's byte b.
+__device__ __forceinline__ void gather_bytes(const uint32_t (&w)[8], int b, uint32_t& lo,
+                                             uint32_t& hi) {
+    const uint32_t sel = (uint32_t)b | ((uint32_t)(4 + b) << 4);
+    const uint32_t p01 = __byte_perm(w[0], w[1], sel), p23 = __byte_perm(w[2], w[3], sel);
+    const uint32_t p45 = __byte_perm(w[4], w[5], sel), p67 = __byte_perm(w[6], w[7], sel);
+    lo = __byte_perm(p01, p23, 0x5410);
+    hi = __byte_perm(p45, p67, 0x5410);
+}
+
+__device__ __forceinline__ uint32_t byte_of(uint32_t lo, uint32_t hi, int c) {
+    return ((c < 4 ? lo : hi) >> (8 * (c & 3))) & 0xffu;
+}
+
 // Block-wide fixed-order sum of one double per warp held by lane 0 in red[warp].
 __device__ __forceinline__ double block_total(const double* red) {
     double t = 0.0;
@@ -172,7 +197,7 @@ struct WorkerArgs {
     const void* g;        // [W][d] caller-owned, GT
     float* ew;            // [W][ld] lazy residual: holds last step's x_w
     const float* s_lazy;  // [W][nch] scale that rebuilds the residual
-    uint32_t* bits_w;     // [W][ldw]
+    uint8_t* sbits;       // [ceil(W/8)][ld] sign bits grouped by 8 workers (single GPU)
     double* part_w;       // [W][nch][nseg]
     uint32_t* status;
     const DpRoute* route;  // data-parallel ranks only: where the plane words go
@@ -231,6 +256,24 @@ template <bool VEC> struct GradLoadN<uint16_t, VEC, 8> {
     }
 };
 
+// Sign bits grouped by 8 workers: byte i of group row g holds the bits of workers 8g .. 8g+7 of
+// element i (bit j = worker 8g + j), the layout the server kernel decodes without transposing.
+// A thread collects, over 8 consecutive workers, its EPT elements' bits -- EPT = 8: byte j of
+// (lo, hi) = worker 8g + j's 8 bits; EPT = 4: nibble j of lo = worker 8g + j's 4 bits -- and
+// transposes them into one byte per element.
+template <int EPT>
+__device__ __forceinline__ void flush_group_bits(uint32_t lo, uint32_t hi, uint8_t* dst) {
+    if constexpr (EPT == 8) {
+        transpose8x8(lo, hi);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+    } else {
+        const uint32_t t = lo & 0x0f0f0f0fu, u = (lo >> 4) & 0x0f0f0f0fu;
+        uint32_t a = __byte_perm(t, u, 0x5140), b = __byte_perm(t, u, 0x7362);
+        transpose8x8(a, b);
+        *reinterpret_cast<uint32_t*>(dst) = a;
+    }
+}
+
 // The kernel is latency-bound on HBM: more warps in flight beat deeper per-thread prefetch
 // (measured on B200). EPT: elements per thread per item, 4 (fp32 gradients: 16-byte loads; 8
 // resident blocks per SM at 32 registers) or 8 (bf16 gradients: 16-byte loads of 8 values; 6
@@ -239,6 +282,8 @@ template <bool VEC> struct GradLoadN<uint16_t, VEC, 8> {
 // LAZY_M: the shared momentum is the decompressed server message of the previous step, m =
 // (bit ? S_k : -S_k), rebuilt here from the server plane instead of read as fp32 (4 bytes per
 // parameter fewer to read, and k_apply need not write it).
+// Single GPU: the sign bits leave grouped by 8 workers (flush_group_bits), one byte per element
+// and group, so that the server reads each element's 8-worker pattern directly.
 // DP: the worker rows are this rank's W / R workers, and the plane words of chunk k go to row
 // (w0 + w) of the receive planes of the rank that serves chunk k (a store to peer memory), so
 // that the exchange of the compressed allreduce travels with the compression itself.
@@ -299,12 +344,14 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
         }
         __syncthreads();
     }
+    uint32_t glo[ITEMS], ghi[ITEMS];   // sign bits of the current group of 8 workers
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) glo[it] = ghi[it] = 0u;
     for (int w = 0; w < W; ++w) {
         const float sp = a.s_lazy[(int64_t)w * a.geo.nch + k];
         const GT* gw = g0 + (int64_t)w * a.geo.d;
         float* ew = a.ew + (int64_t)w * a.geo.ld + base;
-        uint32_t* bw = DP ? dp_bw0[0] + (int64_t)w * dp_bld[0]
-                          : a.bits_w + (int64_t)w * a.geo.ldw + (base >> 5);
+        uint32_t* bw = DP ? dp_bw0[0] + (int64_t)w * dp_bld[0] : nullptr;
         double ss = 0.0;
 #pragma unroll
         for (int it = 0; it < ITEMS; ++it) {
@@ -342,11 +389,26 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k_worker(const Wor
                     st4(ew + off + 4 * h, t4);
                 }
             }
-            // OR the LPW lanes' bit groups of one 32-element word together (LSB-first)
-            uint32_t word = bits << (EPT * sub);
+            if constexpr (DP) {
+                // OR the LPW lanes' bit groups of one 32-element word together (LSB-first)
+                uint32_t word = bits << (EPT * sub);
 #pragma unroll
-            for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(kFull, word, o);
-            if (sub == 0 && nv[it] > 0) bw[q / LPW] = word;
+                for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(kFull, word, o);
+                if (sub == 0 && nv[it] > 0) bw[q / LPW] = word;
+            } else {
+                const int wi = w & 7;
+                if (EPT == 8) {
+                    if (wi < 4) glo[it] |= bits << (8 * wi);
+                    else ghi[it] |= bits << (8 * (wi - 4));
+                } else {
+                    glo[it] |= bits << (4 * wi);
+                }
+                if ((wi == 7 || w == W - 1) && nv[it] > 0) {
+                    flush_group_bits<EPT>(glo[it], ghi[it],
+                                          a.sbits + (int64_t)(w >> 3) * a.geo.ld + base + off);
+                }
+                if (wi == 7) glo[it] = ghi[it] = 0u;
+            }
         }
         ss = warp_sum(ss);
         if (lane == 0) red_w[w * kWarps + warp] = ss;
@@ -470,6 +532,11 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
+// One plain arrival (no transaction bytes) on a barrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
@@ -514,8 +581,11 @@ __global__ void k_selftest_wait(int limit, uint32_t* timed_out) {
 // chunk: it reads the chunk's W scales, picks the decode mode and builds its lookup tables once,
 // then streams its segments. Each segment's W plane rows (at most 528 bytes each) arrive in
 // shared memory by TMA bulk copies counted on a per-stage mbarrier; with two stages the copies
-// of segment t + 2 are in flight while segment t is decoded. Residuals are read and z written
-// with plain 16-byte accesses.
+// of segment t + 2 are in flight while segment t is decoded. Each warp, done with a stage,
+// arrives on the stage's second mbarrier; thread 0 waits for all eight arrivals before it
+// refills the stage, so no block-wide barrier sits in the segment loop and a warp that is ahead
+// goes straight on to the next stage. Residuals are read and z written with plain 16-byte
+// accesses.
 //
 // Decoding. Thread t owns 8 consecutive elements: byte (t % 4) of one 32-element word of every
 // worker's plane. For each group of 8 workers it gathers their 8 bytes (__byte_perm), transposes
@@ -539,7 +609,8 @@ constexpr int kTileRow = kSegWords + 4;    // staged row: the segment's words pl
 
 struct ServerArgs {
     Geometry geo;
-    const uint32_t* bits_w;  // [W][ldw]
+    const uint8_t* sbits;    // [ceil(W/8)][ld] sign bits grouped by 8 workers (single GPU)
+    const uint32_t* bits_w;  // [W][ldw] per-worker receive planes (data-parallel ranks)
     const float* s;          // [W][nch] this step's worker scales
     float* es;               // [ld] lazy server residual: holds last step's z
     const float* S_lazy;     // [nch]
@@ -575,44 +646,35 @@ __host__ __device__ inline size_t server_smem_bytes(int W, int nst) {
          + kWarps * sizeof(double);                             // reduction
 }
 
-// byte i bit c  ->  byte c bit i, on (lo = bytes 0..3, hi = bytes 4..7): three delta swaps of
-// the row/column index bits; the first two stay inside each 32-bit half.
-__device__ __forceinline__ void transpose8x8(uint32_t& lo, uint32_t& hi) {
-    uint32_t t;
-    t = ((lo >> 7) ^ lo) & 0x00AA00AAu;  lo ^= t ^ (t << 7);
-    t = ((hi >> 7) ^ hi) & 0x00AA00AAu;  hi ^= t ^ (t << 7);
-    t = ((lo >> 14) ^ lo) & 0x0000CCCCu; lo ^= t ^ (t << 14);
-    t = ((hi >> 14) ^ hi) & 0x0000CCCCu; hi ^= t ^ (t << 14);
-    t = ((hi << 4) ^ lo) & 0xF0F0F0F0u;  lo ^= t;  hi ^= t >> 4;
-}
-
-// Byte `b` (0..3) of 8 words -> lo/hi whose byte i is word i's byte b.
-__device__ __forceinline__ void gather_bytes(const uint32_t (&w)[8], int b, uint32_t& lo,
-                                             uint32_t& hi) {
-    const uint32_t sel = (uint32_t)b | ((uint32_t)(4 + b) << 4);
-    const uint32_t p01 = __byte_perm(w[0], w[1], sel), p23 = __byte_perm(w[2], w[3], sel);
-    const uint32_t p45 = __byte_perm(w[4], w[5], sel), p67 = __byte_perm(w[6], w[7], sel);
-    lo = __byte_perm(p01, p23, 0x5410);
-    hi = __byte_perm(p45, p67, 0x5410);
-}
-
-__device__ __forceinline__ uint32_t byte_of(uint32_t lo, uint32_t hi, int c) {
-    return ((c < 4 ? lo : hi) >> (8 * (c & 3))) & 0xffu;
-}
-
 template <bool POW2>
 __device__ __forceinline__ float server_average(double acc, double dW, double invW) {
     return __double2float_rn(POW2 ? acc * invW : __ddiv_rn(acc, dW));
 }
 
-// Start the bulk copies of segment j's W plane rows -- and, with STAGE_RES, its residuals after
-// the wpad rows -- into one stage (thread 0 only).
-template <bool STAGE_RES>
+// Start the bulk copies of segment j's sign bits -- grouped (ceil(W/8) rows of kSegS bytes at
+// word offsets 0, kSegS/4, ...), or with PLANES the W per-worker plane rows (kTileRow words
+// apart) -- and, with STAGE_RES, its residuals after wpad * kTileRow words, into one stage
+// (thread 0 only). The grouped rows fit inside the space of the plane rows.
+template <bool STAGE_RES, bool PLANES>
 __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stage, int wpad,
                                              uint64_t* bar, int64_t c0, int64_t clen,
                                              int64_t j) {
     const int64_t base = c0 + j * kSegS;
     const int64_t len = min((int64_t)kSegS, clen - j * kSegS);
+    const uint32_t es_bytes = STAGE_RES ? (uint32_t)(((len + 3) / 4) * 16) : 0u;
+    if constexpr (!PLANES) {
+        // bytes [base, base + round_up(len, 16)) of each group row: base is a multiple of 32
+        // and rows are ld (a multiple of 64) bytes long, so both ends are 16-byte aligned and
+        // inside the row
+        const uint32_t row_bytes = (uint32_t)(((len + 15) / 16) * 16);
+        const int ngroups = wpad / 8;
+        mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)ngroups + es_bytes);
+        for (int g = 0; g < ngroups; ++g)
+            bulk_load(stage + (size_t)g * (kSegS / 4), a.sbits + (int64_t)g * a.geo.ld + base,
+                      row_bytes, bar);
+        if (STAGE_RES) bulk_load(stage + (size_t)wpad * kTileRow, a.es + base, es_bytes, bar);
+        return;
+    }
     const int64_t wbase = base >> 5;
     // words [wbase & ~3, round_up(wbase + ceil(len / 32), 4)) of each row: both ends 16-byte
     // aligned and inside the row (plane rows are padded to a multiple of 4 words)
@@ -620,7 +682,6 @@ __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stag
     const uint32_t row_bytes = (uint32_t)(((lead + (len + 31) / 32 + 3) / 4) * 16);
     // residuals [base, base + round_up(len, 4)): base is a multiple of 32 elements and the
     // buffer is padded to a multiple of 64, so the copy is 16-byte aligned and in bounds
-    const uint32_t es_bytes = STAGE_RES ? (uint32_t)(((len + 3) / 4) * 16) : 0u;
     mbar_arrive_expect_tx(bar, row_bytes * (uint32_t)a.geo.W + es_bytes);
     for (int w = 0; w < a.geo.W; ++w)
         bulk_load(stage + (size_t)w * kTileRow,
@@ -648,7 +709,8 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wpad = (W + 7) & ~7, ngroups = wpad / 8;
     const int nst = server_stages(W, a.geo.nseg_s);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_srv);             // [nst] (<= 2)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_srv);             // [nst] (<= 2): full
+    uint64_t* ebars = reinterpret_cast<uint64_t*>(smem_srv + 32);       // [nst]: stage read
     int* mode_p = reinterpret_cast<int*>(smem_srv + 16);
     int* emin_p = reinterpret_cast<int*>(smem_srv + 20);     // smallest effective exponent
     double* unit_p = reinterpret_cast<double*>(smem_srv + 24);
@@ -664,16 +726,20 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     const double dW = (double)W, invW = 1.0 / (double)W;
 
     if (tid == 0) {
-        for (int st = 0; st < nst; ++st) mbar_init(&bars[st], 1);
+        for (int st = 0; st < nst; ++st) {
+            mbar_init(&bars[st], 1);
+            mbar_init(&ebars[st], kWarps);
+        }
         for (int t = 0; t < nst && t < nseg_blk; ++t)
-            server_issue<STAGE_RES>(a, stages + (size_t)t * stage_words, wpad, &bars[t], c0, clen,
-                                    j0 + t);
+            server_issue<STAGE_RES, BCAST>(a, stages + (size_t)t * stage_words, wpad, &bars[t],
+                                           c0, clen, j0 + t);
     }
     for (int w = tid; w < wpad; w += kThreads)
         sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
-    for (int st = 0; st < nst; ++st)
-        for (int e = W * kTileRow + tid; e < wpad * kTileRow; e += kThreads)
-            stages[(size_t)st * stage_words + e] = 0u;
+    if constexpr (BCAST)
+        for (int st = 0; st < nst; ++st)
+            for (int e = W * kTileRow + tid; e < wpad * kTileRow; e += kThreads)
+                stages[(size_t)st * stage_words + e] = 0u;
     // without STAGE_RES: the first segment's residuals, fetched while the tables are built
     float zp[kSrvItems][kSrvVec];
     int nvs[kSrvItems];
@@ -769,6 +835,9 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     const double unit = *unit_p;
     const float Sp = a.S_lazy[k];
     double ss = 0.0;
+    int consumed = nseg_blk;                      // segments this warp waited for
+    int issued = nst < nseg_blk ? nst : nseg_blk;  // segments whose copies were issued (thread 0)
+    bool issuing = true;
 
     for (int t = 0; t < nseg_blk; ++t) {
         const int st = t % nst;
@@ -803,27 +872,37 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 const int nv = nvs[it];
                 const int wd = q >> 2, bsel = q & 3;       // word within the segment, byte in it
                 const uint32_t* tw = tile + lead + wd;
+                const uint8_t* gb = reinterpret_cast<const uint8_t*>(tile) + off;
+                // group g's pattern: byte c of (lo, hi) = element c's bits of workers 8g .. 8g+7
+                // (bit i = worker 8g + i): read as it is from the grouped rows, or gathered from
+                // the 8 plane rows and transposed
+                auto pattern = [&](int g, uint32_t& lo, uint32_t& hi) {
+                    if constexpr (!BCAST) {
+                        const uint2 u = *reinterpret_cast<const uint2*>(gb + (size_t)g * kSegS);
+                        lo = u.x;
+                        hi = u.y;
+                    } else {
+                        uint32_t wv[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) wv[i] = tw[(g * 8 + i) * kTileRow];
+                        gather_bytes(wv, bsel, lo, hi);
+                        transpose8x8(lo, hi);
+                    }
+                };
                 float y[kSrvVec];
                 if (mode == kModeY) {
-                    uint32_t wv[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) wv[i] = tw[i * kTileRow];
                     uint32_t lo, hi;
-                    gather_bytes(wv, bsel, lo, hi);
-                    transpose8x8(lo, hi);
+                    pattern(0, lo, hi);
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) y[c] = ylut[byte_of(lo, hi, c)];
                 } else if (mode == kModeInt) {
                     int32_t acc[kSrvVec];
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) acc[c] = 0;
+#pragma unroll 2
                     for (int g = 0; g < ngroups; ++g) {
-                        uint32_t wv[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) wv[i] = tw[(g * 8 + i) * kTileRow];
                         uint32_t lo, hi;
-                        gather_bytes(wv, bsel, lo, hi);
-                        transpose8x8(lo, hi);
+                        pattern(g, lo, hi);
                         const int32_t* L = ilut + g * 256;
 #pragma unroll
                         for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
@@ -837,12 +916,8 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
                     for (int g = 0; g < ngroups; ++g) {
-                        uint32_t wv[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) wv[i] = tw[(g * 8 + i) * kTileRow];
                         uint32_t lo, hi;
-                        gather_bytes(wv, bsel, lo, hi);
-                        transpose8x8(lo, hi);
+                        pattern(g, lo, hi);
                         const double* L = lut + g * 256;
 #pragma unroll
                         for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], L[byte_of(lo, hi, c)]);
@@ -850,14 +925,19 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
                 } else {
+                    // worker by worker, in order 0 .. W-1
                     double acc[kSrvVec];
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) acc[c] = 0.0;
-                    for (int w = 0; w < W; ++w) {
-                        const uint32_t byte = tw[w * kTileRow] >> (8 * bsel);
-                        const double sv = sw[w];
+                    for (int g = 0; g < ngroups; ++g) {
+                        uint32_t lo, hi;
+                        pattern(g, lo, hi);
+                        for (int i = 0; i < 8 && 8 * g + i < W; ++i) {
+                            const double sv = sw[8 * g + i];
 #pragma unroll
-                        for (int c = 0; c < kSrvVec; ++c) acc[c] = __dadd_rn(acc[c], ((byte >> c) & 1u) ? sv : -sv);
+                            for (int c = 0; c < kSrvVec; ++c)
+                                acc[c] = __dadd_rn(acc[c], ((byte_of(lo, hi, c) >> i) & 1u) ? sv : -sv);
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) y[c] = server_average<POW2>(acc[c], dW, invW);
@@ -883,20 +963,33 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 if ((lane & 3) == 0 && nv > 0) a.bits_s[wbase + wd] = word;
             }
         }
-        // everyone is done with this stage (or some thread's wait expired: then all leave,
-        // after one more bounded wait for the copies still in flight)
-        if (__syncthreads_or(!landed)) {
-            if (tid == 0) {
-                atomicOr(a.status, kWaitTimeout);
-                for (int u = t; u < nseg_blk && u < t + nst; ++u)
-                    mbar_wait_bounded(&bars[u % nst], (uint32_t)((u / nst) & 1));
-            }
-            return;
+        // this warp is done with the stage: one arrival on its "read" barrier. A warp whose
+        // wait expired does not arrive (the copy may still land), sets the flag and stops.
+        if (!__all_sync(kFull, landed)) {
+            if (lane == 0) atomicOr(a.status, kWaitTimeout);
+            consumed = t;
+            break;
         }
-        if (tid == 0 && t + nst < nseg_blk)
-            server_issue<STAGE_RES>(a, stages + (size_t)st * stage_words, wpad, &bars[st], c0,
-                                    clen, j0 + t + nst);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ebars[st]);
+        // thread 0 refills the stage once all warps have read it (bounded wait; if it expires,
+        // no further copies are issued and the warps waiting for them time out in turn)
+        if (tid == 0 && t + nst < nseg_blk && issuing) {
+            if (mbar_wait_bounded(&ebars[st], parity)) {
+                server_issue<STAGE_RES, BCAST>(a, stages + (size_t)st * stage_words, wpad,
+                                               &bars[st], c0, clen, j0 + t + nst);
+                issued = t + nst + 1;
+            } else {
+                atomicOr(a.status, kWaitTimeout);
+                issuing = false;
+            }
+        }
     }
+    // copies that thread 0 issued and its warp never waited for (only after an expired wait)
+    // must land before the block leaves: one more bounded wait on each, in order
+    if (tid == 0)
+        for (int u = consumed; u < issued; ++u)
+            mbar_wait_bounded(&bars[u % nst], (uint32_t)((u / nst) & 1));
     ss = warp_sum(ss);
     if (lane == 0) red[warp] = ss;
     __syncthreads();
@@ -969,18 +1062,6 @@ __global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
 }
 
 
-// bf16 bit pattern -> the exactly equal fp64 value. Normal values and +-0 by integer ops (the
-// 8-bit exponent rebiased to 11 bits, the 7-bit fraction moved up); subnormal, inf and NaN
-// inputs through the fp32 conversion.
-__device__ __forceinline__ double bf16_to_f64(uint32_t b) {
-    const uint32_t mag = b & 0x7fffu, e = mag >> 7;
-    if (e == 0u || e == 0xffu) {
-        if (mag == 0u) return __hiloint2double((int)((b & 0x8000u) << 16), 0);
-        return (double)__uint_as_float(b << 16);
-    }
-    return __hiloint2double((int)(((b & 0x8000u) << 16) | ((mag << 13) + 0x38000000u)), 0);
-}
-
 // ------------------------------------------------------------------------------------------
 // Warm-up: one full-precision Adam step on the fp64 worker average (LIT-278 note, "What the
 // evidence does not cover": the warm-up phase is plain Adam). No bias correction.
@@ -988,6 +1069,7 @@ __device__ __forceinline__ double bf16_to_f64(uint32_t b) {
 struct WarmupArgs {
     Geometry geo;
     float beta1, omb1, beta2, omb2, eps, lr;
+    float c1, c2;   // bias corrections 1 - beta^t of this step (BC only)
     const void* g;  // [W][d] caller-owned
     float* m;       // [ld]
     float* v;       // [ld]
@@ -996,7 +1078,10 @@ struct WarmupArgs {
 
 // fp64 sum over the W gradient rows (row stride d) of EPT consecutive elements at offset off,
 // nv of them valid, in worker order (bit-exact with the definition); the loads of UNR workers
-// are issued together so that they are in flight at once.
+// are issued together so that they are in flight at once. A bf16 value becomes fp32 by a 16-bit
+// shift and fp64 by the hardware conversion, both exact for every pattern (measured on B200:
+// this keeps the kernel at the copy bandwidth, where widening with integer operations made it
+// issue-bound at 0.74 of it).
 template <typename GT, bool VEC, int EPT>
 __device__ __forceinline__ void worker_grad_sum(const GT* g0, int64_t d, int W, int64_t off,
                                                 int nv, double (&acc)[EPT]) {
@@ -1015,8 +1100,9 @@ __device__ __forceinline__ void worker_grad_sum(const GT* g0, int64_t d, int W, 
                 const uint32_t r[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    acc[2 * h] = __dadd_rn(acc[2 * h], bf16_to_f64(r[h] & 0xffffu));
-                    acc[2 * h + 1] = __dadd_rn(acc[2 * h + 1], bf16_to_f64(r[h] >> 16));
+                    acc[2 * h] = __dadd_rn(acc[2 * h], (double)__uint_as_float(r[h] << 16));
+                    acc[2 * h + 1] = __dadd_rn(acc[2 * h + 1],
+                                               (double)__uint_as_float(r[h] & 0xffff0000u));
                 }
             }
         }
@@ -1040,7 +1126,9 @@ __device__ __forceinline__ void worker_grad_sum(const GT* g0, int64_t d, int W, 
 }
 
 // EPT elements per thread as in k_worker (8 for bf16, 4 for fp32 gradients).
-template <typename GT, bool VEC, int EPT>
+// BC: Adam's optional bias correction -- the step uses m / c1 and v / c2 (m and v are stored
+// uncorrected); off by default, since the pages' step has none.
+template <typename GT, bool VEC, int EPT, bool BC = false>
 __global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
     constexpr int ITEMS = kSeg / (kThreads * EPT);
     int64_t k, j, base, len;
@@ -1072,13 +1160,25 @@ __global__ void __launch_bounds__(kThreads, 4) k_warmup(const WarmupArgs a) {
                 const float gbar = __double2float_rn(__ddiv_rn(acc[4 * h + c], dW));
                 m[c] = __fadd_rn(__fmul_rn(a.beta1, m[c]), __fmul_rn(a.omb1, gbar));
                 v[c] = __fadd_rn(__fmul_rn(a.beta2, v[c]), __fmul_rn(a.omb2, __fmul_rn(gbar, gbar)));
-                const float den = __fadd_rn(__fsqrt_rn(v[c]), a.eps);
-                x[c] = __fsub_rn(x[c], __fmul_rn(a.lr, __fdiv_rn(m[c], den)));
+                const float mh = BC ? __fdiv_rn(m[c], a.c1) : m[c];
+                const float vh = BC ? __fdiv_rn(v[c], a.c2) : v[c];
+                const float den = __fadd_rn(__fsqrt_rn(vh), a.eps);
+                x[c] = __fsub_rn(x[c], __fmul_rn(a.lr, __fdiv_rn(mh, den)));
             }
             st4(a.m + base + o4, m);
             st4(a.v + base + o4, v);
             st4_caller(a.x + base + o4, nv4 >= 4 ? 4 : nv4, x);
         }
+    }
+}
+
+// The freeze after a bias-corrected warm-up: the compression phase continues from the moments
+// the last warm-up step used, m = m / c1, v = v / c2 (i < n).
+__global__ void k_bc_freeze(float* m, float* v, float c1, float c2, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        m[i] = __fdiv_rn(m[i], c1);
+        v[i] = __fdiv_rn(v[i], c2);
     }
 }
 

@@ -1,0 +1,281 @@
+// kernels_zero_one.cuh -- the 0/1 Adam variant's own kernels (codewithpapers.app "0/1 Adam"
+// page, abstract: each Adam step linearised through stale state estimates and their linear
+// correlation, so that 1-bit compression and local steps work together). The compressed
+// allreduce's server stage and the chunk-scale reductions are 1-bit Adam's (kernels.cuh).
+//
+// State per worker w: its momentum m_w and its accumulated update u_w = sum of lr_t * m_w over
+// the steps since the last synchronisation ([W][ld] each), next to the lazy residual of
+// kernels.cuh. Every H-th step ends with a synchronisation, which compresses u_w + e_w with
+// error feedback, runs the server stage and takes the synchronised step
+// x -= ubar / (sqrt(v) + eps); the momentum estimate mbar = ubar / Gamma (Gamma = the sum of
+// the interval's learning rates) becomes every worker's momentum, and u_w restarts at zero.
+// Neither is written: the next step rebuilds mbar = +-fl(S_k / Gamma) from the server plane
+// and takes u_w = 0 (kZoMBar), as the first step after the freeze takes the warm-up momentum
+// (kZoMShared); only the steps in between read and write the per-worker buffers (kZoMWorker).
+#pragma once
+
+#include "kernels.cuh"
+
+namespace onebit {
+
+// where the momentum a step starts from comes from (and whether u_w starts at zero)
+enum ZoSource : int {
+    kZoMShared = 0,  // the shared fp32 momentum (the warm-up m, first step after the freeze);
+                     // u_w = 0
+    kZoMBar = 1,     // mbar = +-fl(S_k / Gamma) by the last synchronisation's server plane; u_w = 0
+    kZoMWorker = 2,  // each worker's own m_w and u_w (steps after a local step)
+};
+
+struct ZoArgs {
+    Geometry geo;
+    float beta1, omb1, lr;
+    int src;                 // ZoSource
+    const float* m;          // [ld] shared momentum (kZoMShared)
+    const uint32_t* bits_s;  // [ldw] last synchronisation's server plane (kZoMBar)
+    const float* S;          // [nch] its server scales (kZoMBar)
+    float gamma_prev;        // its Gamma (kZoMBar)
+    float* mw;               // [W][ld] per-worker momentum
+    float* uw;               // [W][ld] per-worker accumulated update
+    const void* g;           // [W][d] caller-owned, GT
+    float* ew;               // [W][ld] lazy residual: holds the last synchronisation's x_w
+    const float* s_lazy;     // [W][nch] scale that rebuilds the residual
+    uint8_t* sbits;          // [ceil(W/8)][ld] sign bits grouped by 8 workers
+    double* part_w;          // [W][nch][nseg]
+    uint32_t* status;
+};
+
+// One step of every worker for one segment (a block owns a kSeg segment and loops over the W
+// workers, like k_worker). Local step: m_w = b1 m + (1-b1) g_w; u_w += lr m_w, stored. SYNC
+// (the step that ends with a synchronisation): the same m_w and u_w, then x_w = u_w + e_w
+// compressed as in k_worker (sign bits grouped by 8 workers, lazy residual, fp64 partials of the
+// chunk norm); m_w and u_w are not stored, since the synchronisation replaces them.
+template <typename GT, bool VEC, int EPT, bool SYNC>
+__global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k01_worker(const ZoArgs a) {
+    constexpr int ITEMS = kSeg / (kThreads * EPT);
+    constexpr int LPW = 32 / EPT;  // lanes that share one 32-element word of the server plane
+    extern __shared__ double red_w[];  // [W][kWarps] (SYNC)
+    int64_t k, j, base, len;
+    if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int W = a.geo.W;
+    const int sub = lane & (LPW - 1);
+    const int src = a.src;
+
+    // the shared momentum of the block's elements (kZoMShared, kZoMBar), kept in registers
+    float ms[ITEMS][EPT];
+    int nv[ITEMS];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int q = it * kThreads + tid;
+        const int64_t off = (int64_t)q * EPT;
+        const int64_t r = len - off;
+        nv[it] = r <= 0 ? 0 : (r >= EPT ? EPT : (int)r);
+#pragma unroll
+        for (int c = 0; c < EPT; ++c) ms[it][c] = 0.0f;
+        if (nv[it] > 0 && src == kZoMBar) {
+            const float mb = __fdiv_rn(a.S[k], a.gamma_prev);
+            const uint32_t bits = a.bits_s[(base >> 5) + q / LPW] >> (EPT * sub);
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) ms[it][c] = ((bits >> c) & 1u) ? mb : -mb;
+        } else if (nv[it] > 0 && src == kZoMShared) {
+#pragma unroll
+            for (int h = 0; h < EPT / 4; ++h) {
+                float t4[4];
+                ld4(a.m + base + off + 4 * h, t4);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ms[it][4 * h + c] = t4[c];
+            }
+        }
+    }
+    const float b1 = a.beta1, omb1 = a.omb1, lr = a.lr;
+    const GT* g0 = static_cast<const GT*>(a.g) + base;
+    uint32_t glo[ITEMS], ghi[ITEMS];   // SYNC: sign bits of the current group of 8 workers
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) glo[it] = ghi[it] = 0u;
+    for (int w = 0; w < W; ++w) {
+        const float sp = SYNC ? a.s_lazy[(int64_t)w * a.geo.nch + k] : 0.0f;
+        const GT* gw = g0 + (int64_t)w * a.geo.d;
+        float* mwp = a.mw + (int64_t)w * a.geo.ld + base;
+        float* uwp = a.uw + (int64_t)w * a.geo.ld + base;
+        float* ew = a.ew + (int64_t)w * a.geo.ld + base;
+        double ss = 0.0;
+#pragma unroll
+        for (int it = 0; it < ITEMS; ++it) {
+            const int q = it * kThreads + tid;
+            const int64_t off = (int64_t)q * EPT;
+            float gf[EPT], m0[EPT], u0[EPT], xp[EPT];
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) {
+                gf[c] = 0.0f;
+                m0[c] = ms[it][c];
+                u0[c] = 0.0f;
+                xp[c] = 0.0f;
+            }
+            if (nv[it] > 0) {
+                GradLoadN<GT, VEC, EPT>::load(gw + off, nv[it], gf);
+#pragma unroll
+                for (int h = 0; h < EPT / 4; ++h) {
+                    float t4[4];
+                    if (src == kZoMWorker) {
+                        ld4(mwp + off + 4 * h, t4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) m0[4 * h + c] = t4[c];
+                        ld4(uwp + off + 4 * h, t4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) u0[4 * h + c] = t4[c];
+                    }
+                    if (SYNC) {
+                        ld4(ew + off + 4 * h, t4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) xp[4 * h + c] = t4[c];
+                    }
+                }
+            }
+            float mn[EPT], un[EPT];
+#pragma unroll
+            for (int c = 0; c < EPT; ++c) {
+                const bool ok = c < nv[it];
+                mn[c] = ok ? __fadd_rn(__fmul_rn(b1, m0[c]), __fmul_rn(omb1, gf[c])) : 0.0f;
+                un[c] = ok ? __fadd_rn(u0[c], __fmul_rn(lr, mn[c])) : 0.0f;
+            }
+            if constexpr (!SYNC) {
+                if (nv[it] > 0) {
+#pragma unroll
+                    for (int h = 0; h < EPT / 4; ++h) {
+                        const float tm[4] = {mn[4 * h], mn[4 * h + 1], mn[4 * h + 2], mn[4 * h + 3]};
+                        const float tu[4] = {un[4 * h], un[4 * h + 1], un[4 * h + 2], un[4 * h + 3]};
+                        st4(mwp + off + 4 * h, tm);
+                        st4(uwp + off + 4 * h, tu);
+                    }
+                }
+            } else {
+                float x[EPT];
+                uint32_t bits = 0u;
+#pragma unroll
+                for (int c = 0; c < EPT; ++c) {
+                    const float e = __fsub_rn(xp[c], xp[c] >= 0.0f ? sp : -sp);
+                    const float xv = c < nv[it] ? __fadd_rn(un[c], e) : 0.0f;
+                    x[c] = xv;
+                    bits |= (c < nv[it] && xv >= 0.0f) ? (1u << c) : 0u;
+                    ss = __fma_rn((double)xv, (double)xv, ss);   // NaN here marks a NaN x_w
+                }
+                if (nv[it] > 0) {
+#pragma unroll
+                    for (int h = 0; h < EPT / 4; ++h) {
+                        const float t4[4] = {x[4 * h], x[4 * h + 1], x[4 * h + 2], x[4 * h + 3]};
+                        st4(ew + off + 4 * h, t4);
+                    }
+                }
+                const int wi = w & 7;
+                if (EPT == 8) {
+                    if (wi < 4) glo[it] |= bits << (8 * wi);
+                    else ghi[it] |= bits << (8 * (wi - 4));
+                } else {
+                    glo[it] |= bits << (4 * wi);
+                }
+                if ((wi == 7 || w == W - 1) && nv[it] > 0)
+                    flush_group_bits<EPT>(glo[it], ghi[it],
+                                          a.sbits + (int64_t)(w >> 3) * a.geo.ld + base + off);
+                if (wi == 7) glo[it] = ghi[it] = 0u;
+            }
+        }
+        if constexpr (SYNC) {
+            ss = warp_sum(ss);
+            if (lane == 0) red_w[w * kWarps + warp] = ss;
+        }
+    }
+    if constexpr (SYNC) {
+        __syncthreads();
+        bool nan_seen = false;
+        for (int w = tid; w < W; w += kThreads) {
+            const double tot = block_total(red_w + w * kWarps);
+            a.part_w[((int64_t)w * a.geo.nch + k) * a.geo.nseg + j] = tot;
+            nan_seen |= (tot != tot);
+        }
+        if (nan_seen) atomicOr(a.status, kNanWorker);
+    }
+}
+
+// The synchronised step from the server message of the accumulated updates:
+//   ubar = (bit ? S_k : -S_k);  x -= ubar / (sqrt(v) + eps);
+//   refresh:  mbar = ubar / Gamma;  v = b2 v + (1-b2) mbar^2   (after the step, which used the
+//   old v).
+struct ZoApplyArgs {
+    Geometry geo;
+    float eps, gamma, beta2, omb2;
+    int refresh;
+    const uint32_t* bits_s;  // [ldw]
+    const float* S;          // [nch]
+    float* v;                // [ld]
+    float* x;                // [d] caller-owned
+};
+
+__global__ void __launch_bounds__(kThreads) k01_apply(const ZoApplyArgs a) {
+    int64_t k, j, base, len;
+    if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const float S = a.S[k];
+    const int sh = 4 * (lane & 7);
+#pragma unroll
+    for (int it = 0; it < kItems; ++it) {
+        const int q = it * kThreads + tid;
+        const int64_t off = (int64_t)q * kVec;
+        const int nv = valid_of(len, off);
+        if (nv == 0) continue;
+        const uint32_t nib = a.bits_s[(base >> 5) + (q >> 3)] >> sh;
+        float v[4], x[4];
+        ld4(a.v + base + off, v);
+        ld4_caller(a.x + base + off, nv, x);
+#pragma unroll
+        for (int c = 0; c < kVec; ++c) {
+            const float ub = c < nv ? (((nib >> c) & 1u) ? S : -S) : 0.0f;
+            const float den = __fadd_rn(__fsqrt_rn(v[c]), a.eps);
+            x[c] = __fsub_rn(x[c], __fdiv_rn(ub, den));
+            if (a.refresh) {
+                const float mb = __fdiv_rn(ub, a.gamma);
+                v[c] = __fadd_rn(__fmul_rn(a.beta2, v[c]), __fmul_rn(a.omb2, __fmul_rn(mb, mb)));
+            }
+        }
+        st4_caller(a.x + base + off, nv, x);
+        if (a.refresh) st4(a.v + base + off, v);
+    }
+}
+
+// State export: each worker's momentum and accumulated update for elements [i0, i0 + n),
+// rows r < W, into mw_out[W][n] / uw_out[W][n] (either may be null), from whichever form the
+// state is in (src as in ZoArgs).
+__global__ void k01_export(const ZoArgs a, int64_t i0, int64_t n, float* mw_out, float* uw_out) {
+    const int64_t total = (int64_t)a.geo.W * n;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < total;
+         t += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = t / n, i = i0 + (t - r * n);
+        float m, u;
+        if (a.src == kZoMWorker) {
+            m = a.mw[r * a.geo.ld + i];
+            u = a.uw[r * a.geo.ld + i];
+        } else {
+            u = 0.0f;
+            if (a.src == kZoMShared) {
+                m = a.m[i];
+            } else {
+                const float mb = __fdiv_rn(a.S[i / a.geo.C], a.gamma_prev);
+                m = ((a.bits_s[i >> 5] >> (i & 31)) & 1u) ? mb : -mb;
+            }
+        }
+        if (mw_out) mw_out[t] = m;
+        if (uw_out) uw_out[t] = u;
+    }
+}
+
+// Worker w's local model, out[i] = x[i] - u_w[i] / (sqrt(v[i]) + eps), for i < d.
+__global__ void k01_local_model(const float* x, const float* uw, int zero_u, const float* v,
+                                float eps, int64_t d, float* out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < d;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float den = __fadd_rn(__fsqrt_rn(v[i]), eps);
+        const float u = zero_u ? 0.0f : uw[i];
+        out[i] = __fsub_rn(x[i], __fdiv_rn(u, den));
+    }
+}
+
+}  // namespace onebit

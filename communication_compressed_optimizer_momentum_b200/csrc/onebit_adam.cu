@@ -24,6 +24,7 @@
 #include "onebit_adam.h"
 #include "kernels.cuh"
 #include "kernels_dp.cuh"
+#include "kernels_zero_one.cuh"
 
 using namespace onebit;
 
@@ -58,8 +59,8 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 // S_out have no space here (m, v, the server plane and scales live in the exchange region, the
 // worker planes at their servers) and `route` holds the device copy of the rank's route.
 struct Layout {
-    uint64_t route, m, v, es, ew, bits_w, bits_s, s_out, s_lazy, S_out, S_lazy, part_w, part_s,
-        status;
+    uint64_t route, m, v, es, ew, sbits, bits_s, s_out, s_lazy, S_out, S_lazy, part_w, part_s,
+        status, mw, uw;
     uint64_t total;
 };
 
@@ -93,6 +94,17 @@ struct DpState {
 
 }  // namespace
 
+// The 0/1 Adam variant's schedule and step state (zero_one false: a 1-bit Adam handle).
+struct ZoState {
+    bool on = false;
+    int32_t H = 1, K = 0;      // a synchronisation every H steps, a refresh every K-th (0: never)
+    int32_t t = 0;             // steps since the last synchronisation
+    int64_t syncs = 0;
+    float gamma = 0.0f;        // fp32 sum of the learning rates since the last synchronisation
+    float gamma_prev = 0.0f;   // Gamma of the last synchronisation (mbar = ubar / gamma_prev)
+    int src = kZoMShared;      // where the next step's momentum comes from (ZoSource)
+};
+
 struct onebit_adam_s {
     Geometry geo;
     int64_t nw;  // words per plane, ceil(d / 32)
@@ -106,7 +118,8 @@ struct onebit_adam_s {
     // region pointers (valid once bound)
     float *m = nullptr, *v = nullptr, *es = nullptr, *ew = nullptr;
     float *s_out = nullptr, *s_lazy = nullptr, *S_out = nullptr, *S_lazy = nullptr;
-    uint32_t *bits_w = nullptr, *bits_s = nullptr, *status = nullptr;
+    uint8_t* sbits = nullptr;  // worker sign bits grouped by 8 workers (single GPU)
+    uint32_t *bits_s = nullptr, *status = nullptr;
     double *part_w = nullptr, *part_s = nullptr;
     // per-kernel timing
     std::vector<cudaEvent_t> ev;
@@ -117,6 +130,12 @@ struct onebit_adam_s {
     cudaEvent_t step_done = nullptr, d2h_done = nullptr;
     bool d2h_pending = false;
     DpState dp;
+    ZoState zo;
+    // optional bias-corrected warm-up: the fp64 products beta^t of the steps so far
+    bool bc = false;
+    int64_t wsteps = 0;
+    double p1 = 1.0, p2 = 1.0;
+    float *mw = nullptr, *uw = nullptr;  // the 0/1 variant's per-worker momentum and update
 };
 
 namespace {
@@ -139,7 +158,7 @@ Layout make_layout(const onebit_adam_s& h) {
     L.v = take(dp ? 0 : g.ld * f);
     L.es = take(gs.ld * f);
     L.ew = take((uint64_t)g.W * g.ld * f);
-    L.bits_w = take(dp ? 0 : (uint64_t)g.W * g.ldw * u);
+    L.sbits = take(dp ? 0 : (uint64_t)((g.W + 7) / 8) * g.ld);
     L.bits_s = take(dp ? 0 : g.ldw * u);
     L.s_out = take((uint64_t)g.W * g.nch * f);
     L.s_lazy = take((uint64_t)g.W * g.nch * f);
@@ -148,6 +167,8 @@ Layout make_layout(const onebit_adam_s& h) {
     L.part_w = take((uint64_t)g.W * g.nch * g.nseg * sizeof(double));
     L.part_s = take((uint64_t)std::max<int64_t>(gs.nch, 1) * g.nseg_s * sizeof(double));
     L.status = take(4 * sizeof(uint32_t));
+    L.mw = take(h.zo.on ? (uint64_t)g.W * g.ld * f : 0);
+    L.uw = take(h.zo.on ? (uint64_t)g.W * g.ld * f : 0);
     L.total = off;
     return L;
 }
@@ -282,7 +303,7 @@ void launch_worker_t(onebit_adam_s* h, const WorkerArgs& a, unsigned blocks, siz
 template <typename GT>
 int launch_worker(onebit_adam_s* h, const void* grads, cudaStream_t st) {
     WorkerArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->m, h->bits_s, h->S_out, grads, h->ew,
-                 h->s_lazy, h->bits_w, h->part_w, h->status, h->dp.route_dev};
+                 h->s_lazy, h->sbits, h->part_w, h->status, h->dp.route_dev};
     const size_t smem = (size_t)h->geo.W * kWarps * sizeof(double);
     const unsigned blocks = (unsigned)step_blocks(h->geo);
     if (is_dp(h)) {
@@ -310,23 +331,38 @@ int launch_materialize_m(onebit_adam_s* h, int64_t i0, int64_t n, float* dst, cu
     return ONEBIT_OK;
 }
 
-template <typename GT>
-int launch_warmup(onebit_adam_s* h, float* x, const void* grads, float lr, cudaStream_t st) {
-    WarmupArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->beta2, 1.0f - h->beta2, h->eps, lr,
-                 grads, h->m, h->v, x};
+// c_t = fl32(1 - beta^t), beta^t the fp64 product of t factors beta (its fp32 value) in step
+// order: the bias corrections of the optional bias-corrected warm-up (1 - beta2^t would lose
+// most of its digits to cancellation in fp32).
+float bias_correction(double p) { return (float)(1.0 - p); }
+
+template <typename GT, bool BC>
+void launch_warmup_t(onebit_adam_s* h, const WarmupArgs& a, cudaStream_t st) {
     const unsigned blocks = (unsigned)step_blocks(h->geo);
     const int64_t d = h->geo.d;
     if constexpr (sizeof(GT) == 2) {
         if (d % 8 == 0) {
-            k_warmup<GT, true, 8><<<blocks, kThreads, 0, st>>>(a);
-            ONEBIT_CUDA(cudaGetLastError());
-            return ONEBIT_OK;
+            k_warmup<GT, true, 8, BC><<<blocks, kThreads, 0, st>>>(a);
+            return;
         }
     }
     if (d % kVec == 0)
-        k_warmup<GT, true, 4><<<blocks, kThreads, 0, st>>>(a);
+        k_warmup<GT, true, 4, BC><<<blocks, kThreads, 0, st>>>(a);
     else
-        k_warmup<GT, false, 4><<<blocks, kThreads, 0, st>>>(a);
+        k_warmup<GT, false, 4, BC><<<blocks, kThreads, 0, st>>>(a);
+}
+
+template <typename GT>
+int launch_warmup(onebit_adam_s* h, float* x, const void* grads, float lr, cudaStream_t st) {
+    WarmupArgs a{h->geo, h->beta1, 1.0f - h->beta1, h->beta2, 1.0f - h->beta2, h->eps, lr,
+                 1.0f, 1.0f, grads, h->m, h->v, x};
+    if (h->bc) {
+        a.c1 = bias_correction(h->p1 * (double)h->beta1);
+        a.c2 = bias_correction(h->p2 * (double)h->beta2);
+        launch_warmup_t<GT, true>(h, a, st);
+    } else {
+        launch_warmup_t<GT, false>(h, a, st);
+    }
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }
@@ -454,8 +490,8 @@ int dp_compressed_phase(onebit_adam_s* h, int phase, float* x, const void* grads
         if (gs.d > 0) {
             uint32_t* planes = reinterpret_cast<uint32_t*>(dp.xch + dp.xl.planes);
             const float* rs = reinterpret_cast<const float*>(dp.xch + dp.xl.rscales);
-            ServerArgs sa{gs, planes, rs, h->es, h->S_lazy, h->bits_s + dp.e0 / 32, h->part_s,
-                          h->status, dp.route_dev};
+            ServerArgs sa{gs, nullptr, planes, rs, h->es, h->S_lazy, h->bits_s + dp.e0 / 32,
+                          h->part_s, h->status, dp.route_dev};
             const size_t ssm = server_smem_bytes(gs.W, server_stages(gs.W, gs.nseg_s));
             server_kernel_dp(gs.W)<<<(unsigned)server_blocks(gs), kThreads, ssm, st>>>(sa);
             ONEBIT_CUDA(cudaGetLastError());
@@ -555,7 +591,7 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->v = reinterpret_cast<float*>(b + L.v);
     h->es = reinterpret_cast<float*>(b + L.es);
     h->ew = reinterpret_cast<float*>(b + L.ew);
-    h->bits_w = reinterpret_cast<uint32_t*>(b + L.bits_w);
+    h->sbits = reinterpret_cast<uint8_t*>(b + L.sbits);
     h->bits_s = reinterpret_cast<uint32_t*>(b + L.bits_s);
     h->s_out = reinterpret_cast<float*>(b + L.s_out);
     h->s_lazy = reinterpret_cast<float*>(b + L.s_lazy);
@@ -564,6 +600,8 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->part_w = reinterpret_cast<double*>(b + L.part_w);
     h->part_s = reinterpret_cast<double*>(b + L.part_s);
     h->status = reinterpret_cast<uint32_t*>(b + L.status);
+    h->mw = h->zo.on ? reinterpret_cast<float*>(b + L.mw) : nullptr;
+    h->uw = h->zo.on ? reinterpret_cast<float*>(b + L.uw) : nullptr;
     h->gtype = grad_dtype;
     cudaStream_t st = as_stream(stream);
     if (is_dp(h)) {
@@ -579,7 +617,7 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
         h->v = reinterpret_cast<float*>(x + dp.xl.v);
         h->bits_s = reinterpret_cast<uint32_t*>(x + dp.xl.bits_s);
         h->S_out = reinterpret_cast<float*>(x + dp.xl.S);
-        h->bits_w = nullptr;
+        h->sbits = nullptr;
         dp.route_dev = reinterpret_cast<DpRoute*>(b + L.route);
         dp.epoch_dev = reinterpret_cast<uint32_t*>(b + L.route + sizeof(DpRoute));
         dp.connected = false;
@@ -599,6 +637,8 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
     h->phase = kWarmup;
     h->steps = 0;
     h->m_explicit = true;
+    h->wsteps = 0;
+    h->p1 = h->p2 = 1.0;
     return ONEBIT_OK;
 }
 
@@ -618,8 +658,22 @@ int onebit_adam_warmup_step(onebit_adam_t h, float* x, const void* grads, float 
         if (rc == ONEBIT_OK) rc = dp_warmup_phase(h, 2, x, grads, lr, 0, 0, st);
         return rc;
     }
-    return h->gtype == ONEBIT_BF16 ? launch_warmup<uint16_t>(h, x, grads, lr, st)
-                                   : launch_warmup<float>(h, x, grads, lr, st);
+    const int rc = h->gtype == ONEBIT_BF16 ? launch_warmup<uint16_t>(h, x, grads, lr, st)
+                                           : launch_warmup<float>(h, x, grads, lr, st);
+    if (rc == ONEBIT_OK) {
+        ++h->wsteps;
+        h->p1 *= (double)h->beta1;
+        h->p2 *= (double)h->beta2;
+    }
+    return rc;
+}
+
+int onebit_adam_set_bias_correction(onebit_adam_t h, int32_t on) {
+    if (!valid_handle(h) || (on != 0 && on != 1)) return ONEBIT_ERR_ARG;
+    if (is_dp(h)) return ONEBIT_ERR_ARG;
+    if (h->phase == kCompressed || h->wsteps > 0) return ONEBIT_ERR_PHASE;
+    h->bc = on != 0;
+    return ONEBIT_OK;
 }
 
 int onebit_adam_freeze_variance(onebit_adam_t h, void* stream) {
@@ -628,6 +682,13 @@ int onebit_adam_freeze_variance(onebit_adam_t h, void* stream) {
     cudaStream_t st = as_stream(stream);
     const Layout& L = h->lay;
     if (is_dp(h) && h->dp.phase_kind != 0) return ONEBIT_ERR_PHASE;
+    // after a bias-corrected warm-up the compression phase continues from the corrected moments
+    if (h->bc && h->wsteps > 0 && h->geo.d > 0) {
+        const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(h->geo.d, kThreads), 148 * 32);
+        k_bc_freeze<<<blocks, kThreads, 0, st>>>(h->m, h->v, bias_correction(h->p1),
+                                                 bias_correction(h->p2), h->geo.d);
+        ONEBIT_CUDA(cudaGetLastError());
+    }
     // residuals (lazy form: stored 0 with scale 0 rebuilds e = 0), planes, scales, partials
     ONEBIT_CUDA(cudaMemsetAsync(h->ws + L.es, 0, L.total - L.es, st));
     if (is_dp(h)) {
@@ -639,13 +700,20 @@ int onebit_adam_freeze_variance(onebit_adam_t h, void* stream) {
     }
     h->phase = kCompressed;
     h->steps = 0;
+    if (h->zo.on) {
+        ZoState& z = h->zo;
+        z.t = 0;
+        z.syncs = 0;
+        z.gamma = z.gamma_prev = 0.0f;
+        z.src = kZoMShared;  // every worker starts from the warm-up momentum, u_w = 0
+    }
     return ONEBIT_OK;
 }
 
 int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, float lr,
                                 void* stream) {
     if (!valid_handle(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
-    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (h->phase != kCompressed || h->zo.on) return ONEBIT_ERR_PHASE;
     if (h->geo.d == 0) {
         ++h->steps;
         return ONEBIT_OK;
@@ -682,7 +750,8 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
     rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out, h->s_lazy, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 2, st);
-    ServerArgs sa{g, h->bits_w, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s, h->status};
+    ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s,
+                  h->status};
     const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
     const unsigned sblocks = (unsigned)server_blocks(g);
     server_kernel(g.W)<<<sblocks, kThreads, ssm, st>>>(sa);
@@ -706,7 +775,7 @@ int onebit_adam_compressed_step_host(onebit_adam_t h, float* x_dev, void* grads_
                                      const void* grads_host, float* x_host, float lr,
                                      void* stream) {
     if (!valid_handle(h)) return ONEBIT_ERR_ARG;
-    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (h->phase != kCompressed || h->zo.on) return ONEBIT_ERR_PHASE;
     if (h->geo.d == 0) return onebit_adam_compressed_step(h, x_dev, grads_dev, lr, stream);
     if (grads_host == nullptr || x_host == nullptr || grads_dev == nullptr || x_dev == nullptr)
         return ONEBIT_ERR_ARG;
@@ -761,6 +830,7 @@ int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* strea
     int rc = onebit_adam_state_bytes(h, which, &bytes);
     if (rc != ONEBIT_OK) return rc;
     if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
+    if (h->zo.on && which == ONEBIT_STATE_M) return ONEBIT_ERR_ARG;  // per worker: onebit01_*
     if (bytes == 0) return ONEBIT_OK;
     if (dst == nullptr) return ONEBIT_ERR_ARG;
     cudaStream_t st = as_stream(stream);
@@ -775,11 +845,8 @@ int onebit_adam_get_state(onebit_adam_t h, int32_t which, void* dst, void* strea
         case ONEBIT_STATE_SW: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->s_out, bytes, D2D, st)); break;
         case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out, bytes, D2D, st)); break;
         case ONEBIT_STATE_BITSW:
-            if (is_dp(h)) return launch_pack_rows(h, 0, g.d, static_cast<uint32_t*>(dst), st);
-            ONEBIT_CUDA(cudaMemcpy2DAsync(dst, h->nw * sizeof(uint32_t), h->bits_w,
-                                          g.ldw * sizeof(uint32_t), h->nw * sizeof(uint32_t),
-                                          g.W, D2D, st));
-            break;
+            // the signs of the stored x_w (the lazy residual holds x_w itself)
+            return launch_pack_rows(h, 0, g.d, static_cast<uint32_t*>(dst), st);
         case ONEBIT_STATE_BITSS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->bits_s, bytes, D2D, st)); break;
         case ONEBIT_STATE_EW:
         case ONEBIT_STATE_ES: {
@@ -800,6 +867,7 @@ int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void*
     if (h->phase == kUnbound) return ONEBIT_ERR_PHASE;
     const Geometry& g = h->geo;
     if (k < 0 || k >= g.nch || dst == nullptr) return ONEBIT_ERR_ARG;
+    if (h->zo.on && which == ONEBIT_STATE_M) return ONEBIT_ERR_ARG;
     cudaStream_t st = as_stream(stream);
     const int64_t i0 = k * g.C, n = std::min(g.C, g.d - i0);
     const int64_t w0 = i0 / 32, nwk = ceil_div(n, 32);
@@ -827,10 +895,7 @@ int onebit_adam_get_chunk_state(onebit_adam_t h, int32_t which, int64_t k, void*
             break;
         case ONEBIT_STATE_SS: ONEBIT_CUDA(cudaMemcpyAsync(dst, h->S_out + k, f, D2D, st)); break;
         case ONEBIT_STATE_BITSW:
-            if (is_dp(h)) return launch_pack_rows(h, i0, n, static_cast<uint32_t*>(dst), st);
-            ONEBIT_CUDA(cudaMemcpy2DAsync(dst, nwk * u, h->bits_w + w0, g.ldw * u, nwk * u, g.W,
-                                          D2D, st));
-            break;
+            return launch_pack_rows(h, i0, n, static_cast<uint32_t*>(dst), st);
         case ONEBIT_STATE_BITSS:
             ONEBIT_CUDA(cudaMemcpyAsync(dst, h->bits_s + w0, nwk * u, D2D, st));
             break;
@@ -847,6 +912,7 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
     if (which != ONEBIT_STATE_M && which != ONEBIT_STATE_V && which != ONEBIT_STATE_EW &&
         which != ONEBIT_STATE_ES)
         return ONEBIT_ERR_ARG;
+    if (h->zo.on && which != ONEBIT_STATE_V) return ONEBIT_ERR_ARG;
     if (bytes == 0) return ONEBIT_OK;
     if (src == nullptr) return ONEBIT_ERR_ARG;
     cudaStream_t st = as_stream(stream);
@@ -1193,6 +1259,194 @@ int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t
     if (n > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
     k_unpack<<<(unsigned)ceil_div(n, kSeg), kThreads, 0, as_stream(stream)>>>(words, scales, n,
                                                                             C, out);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// The 0/1 Adam variant (codewithpapers.app "0/1 Adam" page, abstract): local steps on each
+// worker's own momentum and accumulated update, and every H-th step a synchronisation through
+// the compressed allreduce of the accumulated updates.
+
+namespace {
+
+template <typename GT, bool SYNC>
+void launch_zo_worker_t(onebit_adam_s* h, const ZoArgs& a, unsigned blocks, size_t smem,
+                        cudaStream_t st) {
+    const int64_t d = h->geo.d;
+    if constexpr (sizeof(GT) == 2) {
+        if (d % 8 == 0) {
+            k01_worker<GT, true, 8, SYNC><<<blocks, kThreads, smem, st>>>(a);
+            return;
+        }
+    }
+    if (d % kVec == 0)
+        k01_worker<GT, true, 4, SYNC><<<blocks, kThreads, smem, st>>>(a);
+    else
+        k01_worker<GT, false, 4, SYNC><<<blocks, kThreads, smem, st>>>(a);
+}
+
+ZoArgs zo_args(onebit_adam_s* h, const void* grads, float lr) {
+    ZoArgs a{};
+    a.geo = h->geo;
+    a.beta1 = h->beta1;
+    a.omb1 = 1.0f - h->beta1;
+    a.lr = lr;
+    a.src = h->zo.src;
+    a.m = h->m;
+    a.bits_s = h->bits_s;
+    a.S = h->S_out;
+    a.gamma_prev = h->zo.gamma_prev;
+    a.mw = h->mw;
+    a.uw = h->uw;
+    a.g = grads;
+    a.ew = h->ew;
+    a.s_lazy = h->s_lazy;
+    a.sbits = h->sbits;
+    a.part_w = h->part_w;
+    a.status = h->status;
+    return a;
+}
+
+int launch_zo_worker(onebit_adam_s* h, const void* grads, float lr, bool sync, cudaStream_t st) {
+    const ZoArgs a = zo_args(h, grads, lr);
+    const unsigned blocks = (unsigned)step_blocks(h->geo);
+    const size_t smem = sync ? (size_t)h->geo.W * kWarps * sizeof(double) : 0;
+    if (h->gtype == ONEBIT_BF16) {
+        if (sync) launch_zo_worker_t<uint16_t, true>(h, a, blocks, smem, st);
+        else launch_zo_worker_t<uint16_t, false>(h, a, blocks, smem, st);
+    } else {
+        if (sync) launch_zo_worker_t<float, true>(h, a, blocks, smem, st);
+        else launch_zo_worker_t<float, false>(h, a, blocks, smem, st);
+    }
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int onebit01_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1, float beta2,
+                  float eps, int32_t H, int32_t K) {
+    if (out == nullptr) return ONEBIT_ERR_ARG;
+    *out = nullptr;
+    if (H < 1 || H > (1 << 20) || K < 0 || K > (1 << 20)) return ONEBIT_ERR_ARG;
+    const int rc = onebit_adam_init(out, d, W, C, beta1, beta2, eps);
+    if (rc != ONEBIT_OK) return rc;
+    (*out)->zo.on = true;
+    (*out)->zo.H = H;
+    (*out)->zo.K = K;
+    return ONEBIT_OK;
+}
+
+int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* stream) {
+    if (!valid_handle(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
+    if (!h->zo.on || h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    ZoState& z = h->zo;
+    const bool sync = z.t + 1 == z.H;
+    const bool refresh = sync && z.K > 0 && (z.syncs + 1) % z.K == 0;
+    const float gamma = z.gamma + lr;  // fp32, in step order
+    if (h->geo.d > 0) {
+        if (x == nullptr || grads == nullptr) return ONEBIT_ERR_ARG;
+        if (!aligned16(x) || !aligned16(grads)) return ONEBIT_ERR_ALIGN;
+        if (sync && !(gamma != 0.0f && std::isfinite(gamma))) return ONEBIT_ERR_ARG;
+        cudaStream_t st = as_stream(stream);
+        const Geometry& g = h->geo;
+        struct Range {
+            Range() { nvtxRangePushA("onebit01_step"); }
+            ~Range() { nvtxRangePop(); }
+        } range;
+        record(h, 0, st);
+        int rc = launch_zo_worker(h, grads, lr, sync, st);
+        if (rc != ONEBIT_OK) return rc;
+        record(h, 1, st);
+        if (sync) {
+            rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out,
+                               h->s_lazy, st);
+            if (rc != ONEBIT_OK) return rc;
+        }
+        record(h, 2, st);
+        if (sync) {
+            ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s,
+                          h->part_s, h->status};
+            const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
+            server_kernel(g.W)<<<(unsigned)server_blocks(g), kThreads, ssm, st>>>(sa);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+        record(h, 3, st);
+        if (sync) {
+            rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
+                               kSegS * kSrvSegsPerBlock, h->S_out, h->S_lazy, st);
+            if (rc != ONEBIT_OK) return rc;
+        }
+        record(h, 4, st);
+        if (sync) {
+            ZoApplyArgs pa{g, h->eps, gamma, h->beta2, 1.0f - h->beta2, refresh ? 1 : 0,
+                           h->bits_s, h->S_out, h->v, x};
+            k01_apply<<<(unsigned)step_blocks(g), kThreads, 0, st>>>(pa);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+        record(h, 5, st);
+        if (h->tcount < h->tmax) ++h->tcount;
+    }
+    ++h->steps;
+    if (sync) {
+        z.gamma_prev = gamma;
+        z.gamma = 0.0f;
+        z.t = 0;
+        ++z.syncs;
+        z.src = kZoMBar;
+    } else {
+        z.gamma = gamma;
+        ++z.t;
+        z.src = kZoMWorker;
+    }
+    return ONEBIT_OK;
+}
+
+int onebit01_info(onebit_adam_t h, int64_t out[6]) {
+    if (!valid_handle(h) || out == nullptr || !h->zo.on) return ONEBIT_ERR_ARG;
+    const ZoState& z = h->zo;
+    out[0] = z.H;
+    out[1] = z.K;
+    out[2] = z.t;
+    out[3] = z.syncs;
+    out[4] = z.src;
+    out[5] = z.t + 1 == z.H ? kLaunchesPerStep : 1;
+    return ONEBIT_OK;
+}
+
+int onebit01_get_worker_state(onebit_adam_t h, int32_t which, int64_t k, void* dst,
+                              void* stream) {
+    if (!valid_handle(h) || !h->zo.on || dst == nullptr) return ONEBIT_ERR_ARG;
+    if (which != 0 && which != 1) return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    const Geometry& g = h->geo;
+    if (k < -1 || k >= g.nch) return ONEBIT_ERR_ARG;
+    const int64_t i0 = k < 0 ? 0 : k * g.C, n = k < 0 ? g.d : std::min(g.C, g.d - i0);
+    const int64_t total = (int64_t)g.W * n;
+    if (total == 0) return ONEBIT_OK;
+    const ZoArgs a = zo_args(h, nullptr, 0.0f);
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(total, kThreads), 148 * 32);
+    float* out = static_cast<float*>(dst);
+    k01_export<<<blocks, kThreads, 0, as_stream(stream)>>>(a, i0, n, which == 0 ? out : nullptr,
+                                                           which == 1 ? out : nullptr);
+    ONEBIT_CUDA(cudaGetLastError());
+    return ONEBIT_OK;
+}
+
+int onebit01_local_model(onebit_adam_t h, int32_t w, const float* x, float* out, void* stream) {
+    if (!valid_handle(h) || !h->zo.on || x == nullptr || out == nullptr) return ONEBIT_ERR_ARG;
+    const Geometry& g = h->geo;
+    if (w < 0 || w >= g.W) return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (g.d == 0) return ONEBIT_OK;
+    const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(g.d, kThreads), 148 * 32);
+    k01_local_model<<<blocks, kThreads, 0, as_stream(stream)>>>(
+        x, h->uw + (int64_t)w * g.ld, h->zo.src != kZoMWorker, h->v, h->eps, g.d, out);
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }

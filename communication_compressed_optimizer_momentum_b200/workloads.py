@@ -81,6 +81,26 @@ class Workload:
         scales are negligible). (W / R + 1) * d * (R - 1) / (8 R)."""
         return (self.W / R + 1) * self.d * (R - 1) / (8.0 * R)
 
+    def zero_one_bytes_per_param(self, H: int, K: int) -> float:
+        """The 0/1 Adam variant's minimum HBM bytes per parameter per step, averaged over one
+        interval of H steps (a synchronisation every H steps, a variance refresh at every K-th
+        one). The first step after a synchronisation rebuilds the shared momentum estimate from
+        the server plane (1/8) and writes every worker's momentum and accumulated update
+        (W*(G + 8)); the steps in between read and write both (W*(G + 16)); the synchronising
+        step reads them, compresses u_w + e_w (residual read and written, sign plane written:
+        W*(G + 16.125)), then the server stage (W/8 + 8.125) and the synchronised step (server
+        plane, v, x: 12.125, plus 4 when v is refreshed). With H = 1 every step is the 1-bit
+        Adam step's bytes."""
+        G, W = self.grad_bytes, self.W
+        server = W / 8.0 + 8.125
+        apply = 12.125 + (4.0 / K if K > 0 else 0.0)
+        if H == 1:
+            return W * (G + 8.125) + 0.125 + server + apply
+        first = W * (G + 8.0) + 0.125
+        middle = (H - 2) * W * (G + 16.0)
+        sync = W * (G + 16.125) + server + apply
+        return (first + middle + sync) / H
+
     def kernel_bytes_per_param(self) -> dict:
         """The same minimum, split by the three streaming kernels of the step."""
         G, W = self.grad_bytes, self.W

@@ -103,11 +103,24 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
  * One full-precision Adam warm-up step (LIT-278 note, "What the evidence does not cover": the
  * warm-up runs uncompressed Adam). grads: [W][d] of the bound type, device; x: fp32[d], device,
  * updated in place. gbar = fp64 average over workers rounded once; m = b1 m + (1-b1) gbar;
- * v = b2 v + (1-b2) gbar^2; x -= lr * (m / (sqrt(v) + eps)); no bias correction.
- * ONEBIT_ERR_PHASE after onebit_adam_freeze_variance.
+ * v = b2 v + (1-b2) gbar^2; x -= lr * (m / (sqrt(v) + eps)); no bias correction unless
+ * onebit_adam_set_bias_correction turned it on. ONEBIT_ERR_PHASE after
+ * onebit_adam_freeze_variance.
  */
 int onebit_adam_warmup_step(onebit_adam_t h, float* x, const void* grads, float lr,
                             void* stream);
+
+/*
+ * Optional bias-corrected warm-up (off by default: the pages' step x - lr * m / (sqrt(v) + eps)
+ * has no bias correction, and neither page mentions one). With on = 1, warm-up step t uses
+ * Adam's corrected moments m / c1_t and v / c2_t in its step (m and v are stored uncorrected),
+ * c_t = fl32(1 - beta^t) with beta^t the fp64 product of t factors beta (the fp32 value) in
+ * order; onebit_adam_freeze_variance then continues from the corrected moments, m / c1_T and
+ * v / c2_T, so that the first compressed step does not jump in size. Allowed before the first
+ * warm-up step only (ONEBIT_ERR_PHASE afterwards); ONEBIT_ERR_ARG for on not in {0, 1} or a
+ * data-parallel rank's handle. Host only.
+ */
+int onebit_adam_set_bias_correction(onebit_adam_t h, int32_t on);
 
 /*
  * End the warm-up: v becomes the fixed preconditioner ("1-bit Adam" index page, Abstract;
@@ -382,6 +395,77 @@ int onebit_dp_warmup_phase(onebit_adam_t h, int32_t phase, float* x, const void*
                            float lr, void* stream);
 int onebit_dp_compressed_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads,
                                float lr, void* stream);
+
+/*
+ * ------------------------------------------------------------------------------------------
+ * The 0/1 Adam variant (codewithpapers.app "0/1 Adam" page, abstract: each Adam step is
+ * linearised by approximating the optimizer states with their stale estimates and their linear
+ * correlation, which lets 1-bit compression and local steps be used together).
+ *
+ * The page gives no formulas; the library follows these readings (the oracle's Z1-Z7):
+ *   - the warm-up (onebit_adam_warmup_step) and the freeze (onebit_adam_freeze_variance) are
+ *     1-bit Adam's;
+ *   - every step, each worker w takes a local step on its own momentum and accumulated update:
+ *         m_w = beta1*m_w + (1-beta1)*g_w ;  u_w = u_w + lr*m_w
+ *   - every H-th step ends with a synchronisation: 1-bit Adam's compressed allreduce of
+ *     u_w + e_w (per-chunk scale, signs, worker and server error feedback) gives ubar; then
+ *         x = x - ubar / (sqrt(v) + eps) ;  mbar = ubar / Gamma
+ *     with Gamma the fp32 sum of the interval's learning rates (the momentum estimate: u is
+ *     linear in the momenta); every worker restarts from m_w = mbar, u_w = 0;
+ *   - at every K-th synchronisation (K = 0: never) the stale variance is refreshed after the
+ *     step: v = beta2*v + (1-beta2)*mbar^2;
+ *   - worker w's local model between synchronisations is x - u_w / (sqrt(v) + eps).
+ * With H = 1, K = 0 and a power-of-two lr the variant gives 1-bit Adam's parameters bit for bit.
+ * A 0/1 handle is a single-GPU handle: the data-parallel entry points do not apply to it, and
+ * onebit_adam_compressed_step(_host) returns ONEBIT_ERR_PHASE on it.
+ */
+
+/*
+ * Create a 0/1 Adam handle: the arguments and checks of onebit_adam_init, plus the
+ * synchronisation interval H (1 <= H <= 2^20) and the variance refresh period K in
+ * synchronisations (0 <= K <= 2^20; 0 = never). Its workspace (onebit_adam_workspace_bytes)
+ * also holds every worker's momentum and accumulated update, fp32[W][d] each. Host only;
+ * ONEBIT_ERR_ARG for H or K out of range (*out is then NULL).
+ */
+int onebit01_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                  float beta2, float eps, int32_t H, int32_t K);
+
+/*
+ * One step of the variant's compression phase on `stream`: the local step of every worker
+ * (one launch), and on every H-th step the synchronisation as well (four more launches: the
+ * worker scales, 1-bit Adam's server stage, the server scales, the synchronised step), which
+ * updates x (fp32[d], device, in/out). grads is [W][d] (device), fp32 or bf16 as bound.
+ * ONEBIT_ERR_PHASE before the freeze or on a 1-bit Adam handle; ONEBIT_ERR_ARG for a NULL
+ * pointer, a non-finite lr, or a synchronisation whose Gamma is 0 or not finite;
+ * ONEBIT_ERR_ALIGN for pointers that are not 16-byte aligned. The sign planes, scales and
+ * residuals of the last synchronisation are read with onebit_adam_get_state /
+ * onebit_adam_get_chunk_state (not ONEBIT_STATE_M, which a 0/1 handle does not hold).
+ */
+int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* stream);
+
+/*
+ * out[0..5] = H, K, steps since the last synchronisation, synchronisations so far, where the
+ * next step's momentum comes from (0: the warm-up momentum, 1: the last synchronisation's
+ * mbar, 2: each worker's own), launches of the next step (5 when it synchronises, else 1).
+ * Host only; ONEBIT_ERR_ARG for a 1-bit Adam handle.
+ */
+int onebit01_info(onebit_adam_t h, int64_t out[6]);
+
+/*
+ * Every worker's momentum (which = 0) or accumulated update (which = 1) into dst (device):
+ * fp32[W][d] for k = -1, fp32[W][C_k] for chunk k. Queued on `stream`. ONEBIT_ERR_ARG for a
+ * 1-bit Adam handle, which not in {0, 1}, k out of range or a NULL dst; ONEBIT_ERR_PHASE
+ * before the freeze.
+ */
+int onebit01_get_worker_state(onebit_adam_t h, int32_t which, int64_t k, void* dst,
+                              void* stream);
+
+/*
+ * Worker w's local model x - u_w / (sqrt(v) + eps) into out (fp32[d], device), with x the
+ * synchronised parameters (fp32[d], device). ONEBIT_ERR_ARG for a 1-bit Adam handle, w out of
+ * range or a NULL pointer; ONEBIT_ERR_PHASE before the freeze.
+ */
+int onebit01_local_model(onebit_adam_t h, int32_t w, const float* x, float* out, void* stream);
 
 /* Static description of a status code. */
 const char* onebit_strerror(int32_t code);

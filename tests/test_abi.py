@@ -16,7 +16,7 @@ HEADER = os.path.join(ROOT, "include", "onebit_adam.h")
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"\b(onebit_\w+)\s*\(", text)
+    names = re.findall(r"\b(onebit\w*)\s*\(", text)
     return sorted(set(names))
 
 
@@ -137,3 +137,57 @@ def test_strerror_covers_codes(lib):
     for c in (0, -1, -2, -3, -4, -5):
         assert lib.onebit_strerror(c).decode() != "unknown status"
     assert lib.onebit_strerror(12345).decode() == "unknown status"
+
+
+def test_zero_one_entry_points_validate_on_the_host(lib):
+    """The 0/1 Adam variant's entry points reject bad arguments and wrong handles before any
+    device work."""
+    h = ctypes.c_void_p()
+    assert lib.onebit01_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8, 0, 1) == -1
+    assert h.value is None
+    assert lib.onebit01_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8, 4, -1) == -1
+    assert lib.onebit01_init(ctypes.byref(h), 1000, 4, 100, 0.9, 0.999, 1e-8, 4, 1) == -2
+    assert lib.onebit01_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8, 4, 2) == 0
+    info = (ctypes.c_int64 * 6)()
+    assert lib.onebit01_info(h, info) == 0
+    assert list(info)[:4] == [4, 2, 0, 0]
+    # unbound: no step, no state
+    assert lib.onebit01_step(h, None, None, ctypes.c_float(1e-3), None) == -3
+    assert lib.onebit01_get_worker_state(h, 0, -1, ctypes.c_void_p(0x1000), None) == -3
+    assert lib.onebit01_get_worker_state(h, 2, -1, ctypes.c_void_p(0x1000), None) == -1
+    assert lib.onebit01_local_model(h, 4, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000),
+                                    None) == -1
+    lib.onebit_adam_destroy(h)
+    # a 1-bit Adam handle is not a 0/1 handle
+    one = ctypes.c_void_p()
+    assert lib.onebit_adam_init(ctypes.byref(one), 1000, 4, 256, 0.9, 0.999, 1e-8) == 0
+    assert lib.onebit01_info(one, info) == -1
+    assert lib.onebit01_step(one, None, None, ctypes.c_float(1e-3), None) == -3
+    lib.onebit_adam_destroy(one)
+
+
+def test_zero_one_workspace_holds_per_worker_state(lib):
+    a, b = ctypes.c_void_p(), ctypes.c_void_p()
+    d, W = 100_000, 4
+    assert lib.onebit_adam_init(ctypes.byref(a), d, W, 4096, 0.9, 0.999, 1e-8) == 0
+    assert lib.onebit01_init(ctypes.byref(b), d, W, 4096, 0.9, 0.999, 1e-8, 4, 0) == 0
+    na, nb = ctypes.c_uint64(), ctypes.c_uint64()
+    assert lib.onebit_adam_workspace_bytes(a, 0, ctypes.byref(na)) == 0
+    assert lib.onebit_adam_workspace_bytes(b, 0, ctypes.byref(nb)) == 0
+    ld = (d + 63) // 64 * 64
+    assert nb.value - na.value >= 2 * W * ld * 4        # m_w and u_w, fp32[W][d] each
+    lib.onebit_adam_destroy(a)
+    lib.onebit_adam_destroy(b)
+
+
+def test_bias_correction_switch_validates_on_the_host(lib):
+    h = ctypes.c_void_p()
+    assert lib.onebit_adam_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8) == 0
+    assert lib.onebit_adam_set_bias_correction(h, 2) == -1
+    assert lib.onebit_adam_set_bias_correction(h, 1) == 0
+    assert lib.onebit_adam_set_bias_correction(h, 0) == 0
+    lib.onebit_adam_destroy(h)
+    r = ctypes.c_void_p()
+    assert lib.onebit_dp_init(ctypes.byref(r), 1000, 4, 256, 0.9, 0.999, 1e-8, 2, 0) == 0
+    assert lib.onebit_adam_set_bias_correction(r, 1) == -1      # single-GPU handles only
+    lib.onebit_adam_destroy(r)
