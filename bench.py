@@ -79,7 +79,10 @@ def get_workload(name, scale_d=0):
     if name.startswith("sweep_W"):
         # sweep_W<w>_C<c>, c = 0 for d/W
         w, c = name[len("sweep_W"):].split("_C")
-        return wls.sweep_workload(int(w), int(c) or None)
+        wl = wls.sweep_workload(int(w), int(c) or None)
+        if scale_d:
+            wl = wls.scaled(wl, scale_d, C=None if not int(c) else min(int(c), scale_d))
+        return wl
     raise SystemExit("unknown workload %s" % name)
 
 

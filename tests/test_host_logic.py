@@ -126,3 +126,12 @@ def test_clock_sampler_parses_nvidia_smi_lines():
 
 def test_whole_job_rate():
     assert bench.whole_job_rate(1000, 4, 2.0) == pytest.approx(4000 / 0.002)
+
+
+def test_scaled_sweep_workloads_for_profiling():
+    """--scale-d shrinks the sweep points too (ncu captures must stay a few GB)."""
+    wl = bench.get_workload("sweep_W64_C0", 1 << 24)
+    assert (wl.d, wl.W, wl.C) == (1 << 24, 64, (1 << 24) // 64)
+    wl = bench.get_workload("sweep_W64_C4096", 1 << 24)
+    assert (wl.d, wl.C) == (1 << 24, 4096)
+    assert bench.get_workload("sweep_W2_C0").d == 1 << 28
