@@ -66,9 +66,19 @@ def parse_args():
     p.add_argument("--sync-every", type=int, default=4, help="0/1 Adam: H")
     p.add_argument("--refresh-every", type=int, default=2,
                    help="0/1 Adam: variance refresh every K-th synchronisation (0: never)")
+    p.add_argument("--kernel-events", default="inline", choices=("inline", "separate"),
+                   help="inline: the per-kernel CUDA events are recorded inside the timed "
+                        "region; separate: the timed region runs without them and the "
+                        "per-kernel times come from a second pass of the same length (for "
+                        "launch-bound small workloads, where recording events costs host time)")
     p.add_argument("--no-dp-section", action="store_true",
                    help="under torchrun with N > 1, skip timing the data-parallel step after "
                         "the replica headline")
+    p.add_argument("--write-traffic", metavar="CSV",
+                   help="write the DRAM traffic summary from an ncu CSV captured with "
+                        "--scale-d on the current kernels, then exit (no GPU needed)")
+    p.add_argument("--traffic-command", default="",
+                   help="with --write-traffic: the ncu command line that made the CSV")
     return p.parse_args()
 
 
@@ -120,6 +130,57 @@ def ncu_traffic(workload):
         except (KeyError, TypeError, ValueError):
             continue
     return out
+
+
+def write_traffic_json(csv_path, workload, captured_params, command, out=TRAFFIC_JSON):
+    """Writes the DRAM traffic summary that ncu_traffic reads, from the CSV of an
+    ``ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum --csv``
+    capture of the step's kernels on a ``--scale-d captured_params`` copy of the workload. The
+    last captured launch of each kernel (a steady-state step) is kept; every stream of the three
+    kernels is per parameter, so its bytes scale to the full workload by d / captured_params."""
+    import csv
+    import re
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    rows = list(csv.DictReader(lines))
+    launches = {}
+    for r in rows:
+        m = re.search(r"\bk_(worker|server|apply)\b", r["Kernel Name"])
+        if not m:
+            continue
+        launches.setdefault(m.group(1), {}).setdefault(int(r["ID"]), {})[r["Metric Name"]] = \
+            float(r["Metric Value"].replace(",", ""))
+    wl = get_workload(workload)
+    kb = wl.kernel_bytes_per_param()
+    scale = wl.d / captured_params
+    kernels = {}
+    for name in ("worker", "server", "apply"):
+        if name not in launches:
+            raise SystemExit("no k_%s launch in %s" % (name, csv_path))
+        met = launches[name][max(launches[name])]
+        rd, wr = met["dram__bytes_read.sum"], met["dram__bytes_write.sum"]
+        alg = kb[name] * captured_params
+        kernels[name] = {"dram_bytes_read": int(rd), "dram_bytes_write": int(wr),
+                         "duration_ns": int(met["gpu__time_duration.sum"]),
+                         "algorithmic_bytes_per_param": kb[name], "algorithmic_bytes": alg,
+                         "dram_over_algorithmic": round((rd + wr) / alg, 4),
+                         "dram_bytes_per_launch_full": int(round((rd + wr) * scale))}
+    j = {"workload": workload, "kernel_source_sha256": kernel_source_sha(),
+         "capture": {"command": command, "captured_params": captured_params,
+                     "full_params": wl.d, "scale": scale,
+                     "note": "one launch of each kernel of a steady-state compressed step on a "
+                             "smaller copy of the workload; every stream of the three kernels "
+                             "is per parameter, so the bytes scale to the full workload by "
+                             "full_params / captured_params. When the smaller copy's sign bytes "
+                             "and server plane fit the 126 MB L2, the server and apply kernels "
+                             "read part of their input from L2 and their DRAM/algorithmic ratio "
+                             "is a lower bound for the full size. The server kernel's table "
+                             "layout depends on the grid and can differ between the copy and "
+                             "the full size; it changes no DRAM stream."},
+         "kernels": kernels}
+    with open(out, "w") as f:
+        json.dump(j, f, indent=1)
+    return j
 
 
 class ClockSampler:
@@ -412,7 +473,8 @@ def run_ours(args):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.5)
-    opt.timing(0 if graph is not None else args.steps)
+    inline_events = graph is None and args.kernel_events == "inline"
+    opt.timing(args.steps if inline_events else 0)
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -431,6 +493,12 @@ def run_ours(args):
     if world > 1:
         dist.barrier()
     ms = t_start.elapsed_time(t_end)
+    if graph is None and not inline_events:
+        # the same number of steps again, eager, with the per-kernel events
+        opt.timing(args.steps)
+        for _ in range(args.steps):
+            opt.step(x, g, wl.lr)
+        torch.cuda.synchronize()
     kernel_ms, nrec = opt.timing_read()
     opt.timing(0)
     time.sleep(0.3)
@@ -504,7 +572,10 @@ def run_ours(args):
                                (opt.workspace_bytes + wl.W * wl.d * wl.grad_bytes
                                 + wl.d * 4) / 1e9),
                            grads_resident="one seeded draw reused by every timed step",
-                           cuda_graph=bool(args.graph)),
+                           cuda_graph=bool(args.graph),
+                           kernel_events=("none (graph replay)" if args.graph else
+                                          "inside the timed region" if inline_events else
+                                          "separate pass after the timed region")),
             "achieved_hbm_gbs": achieved_step_gbs,
             "pct_of_hbm_peak": 100.0 * achieved_step_gbs / peak,
             "pct_of_nominal_hbm": 100.0 * achieved_step_gbs / NOMINAL_HBM_GBS,
@@ -534,7 +605,9 @@ def run_ours(args):
                             "peak_source": peak_src, "unit": "GB/s",
                             "frac": achieved_step_gbs / peak, "traffic": None,
                             "algorithmic_bytes_per_launch": step_bytes}
-        line["gpu_launches"] = args.steps + 4 * (args.steps // args.sync_every)
+        H, w0 = args.sync_every, max(args.warmup, 0)
+        syncs = (w0 + args.steps) // H - w0 // H       # synchronising steps among the timed ones
+        line["gpu_launches"] = args.steps + 4 * syncs
     opt.close()
     if world > 1:
         # after the replica headline, the same workload as data-parallel ranks: one rank per
@@ -765,7 +838,13 @@ def run_reference(args):
 
 def main():
     args = parse_args()
-    if args.impl == "reference":
+    if args.write_traffic:
+        if not args.scale_d:
+            raise SystemExit("--write-traffic needs the --scale-d the capture ran with")
+        j = write_traffic_json(args.write_traffic, args.workload, args.scale_d,
+                               args.traffic_command)
+        print(json.dumps({k: v["dram_over_algorithmic"] for k, v in j["kernels"].items()}))
+    elif args.impl == "reference":
         run_reference(args)
     elif args.dp:
         run_dp(args)

@@ -16,6 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libonebit_adam.so")
 SOURCES = [os.path.join(SRC_DIR, "onebit_adam.cu")]
 DEPS = SOURCES + [os.path.join(SRC_DIR, "kernels.cuh"), os.path.join(SRC_DIR, "kernels_dp.cuh"),
+                  os.path.join(SRC_DIR, "kernels_zero_one.cuh"),
                   os.path.join(INCLUDE, "onebit_adam.h")]
 
 # --fmad=false: no contraction of the method's fp32 multiply-adds (every fp32 operation is one

@@ -49,6 +49,7 @@ struct Geometry {
     int64_t ld;    // row length (elements) of the library's fp32 [W][ld] residual buffer
     int64_t ldw;   // row length (words) of a packed sign plane
     int32_t W;     // workers
+    int32_t spb;   // server segments per block (server_segs_per_block)
 };
 
 // ------------------------------------------------------------------------------------------
@@ -577,22 +578,23 @@ __global__ void k_selftest_wait(int limit, uint32_t* timed_out) {
 //   store z (lazy server residual);  fp64 partial of sum z^2.
 // LIT-278 note, Key takeaways and "What the evidence does not cover" (the compressed allreduce).
 //
-// Work split. A block owns up to kSrvSegsPerBlock consecutive kSegS-element segments of one
-// chunk: it reads the chunk's W scales, picks the decode mode and builds its lookup tables once,
-// then streams its segments. Each segment's W plane rows (at most 528 bytes each) arrive in
-// shared memory by TMA bulk copies counted on a per-stage mbarrier; with two stages the copies
-// of segment t + 2 are in flight while segment t is decoded. Each warp, done with a stage,
-// arrives on the stage's second mbarrier; thread 0 waits for all eight arrivals before it
-// refills the stage, so no block-wide barrier sits in the segment loop and a warp that is ahead
-// goes straight on to the next stage. Residuals are read and z written with plain 16-byte
-// accesses.
+// Work split. A block owns up to spb (8 or 16) consecutive kSegS-element segments of one chunk:
+// it reads the chunk's W scales, picks the decode mode and builds its lookup tables once, then
+// streams its segments. Each segment's sign bits arrive in shared memory by TMA bulk copies
+// counted on a per-stage mbarrier: on one GPU the ceil(W/8) rows of the grouped sign bytes
+// (4096 bytes each), on a data-parallel rank the W per-worker plane rows (at most 528 bytes
+// each). With two stages the copies of segment t + 2 are in flight while segment t is decoded.
+// Each warp, done with a stage, arrives on the stage's second mbarrier; thread 0 waits for all
+// eight arrivals before it refills the stage, so no block-wide barrier sits in the segment loop
+// and a warp that is ahead goes straight on to the next stage. Residuals are staged with the
+// sign bits or read into registers, and z is written with plain 16-byte accesses.
 //
-// Decoding. Thread t owns 8 consecutive elements: byte (t % 4) of one 32-element word of every
-// worker's plane. For each group of 8 workers it gathers their 8 bytes (__byte_perm), transposes
-// the 8x8 bit block so that byte c holds element c's 8 worker bits, and looks the 8-bit pattern
-// up in a per-block table of the sums of (+-s) over that group. Every partial sum of the W
-// values +-s_w is exact in fp64 when sum |s_w| <= 2^53 * u (u = the smallest ulp among the
-// nonzero s_w), so then the grouping cannot change the result. The block picks one of four
+// Decoding. Thread t owns 8 consecutive elements. For each group of 8 workers it takes their
+// 8-bit patterns of those elements -- one 8-byte shared load of the grouped sign bytes, or, from
+// per-worker planes, a gather of 8 bytes (__byte_perm) and an 8x8 bit transpose -- and looks
+// each pattern up in a per-block table of the sums of (+-s) over that group. Every partial sum
+// of the W values +-s_w is exact in fp64 when sum |s_w| <= 2^53 * u (u = the smallest ulp among
+// the nonzero s_w), so then the grouping cannot change the result. The block picks one of four
 // decodes, all bit-identical to the in-order fp64 sum of the definition:
 //   kModeY     W <= 8: one table of y itself (its entries are the in-order sums);
 //   kModeInt   exact and sum |s_w| / u < 2^31: the +-s_w are integers in units of u, the tables
@@ -602,7 +604,6 @@ __global__ void k_selftest_wait(int limit, uint32_t* timed_out) {
 
 enum ServerMode : int { kModeY = 0, kModeInt = 1, kModeF64 = 2, kModeSeq = 3 };
 
-constexpr int kSrvSegsPerBlock = 8;        // server segments per block
 constexpr int kSegWords = kSegS / 32;      // sign words per worker per server segment
 constexpr int kTileRow = kSegWords + 4;    // staged row: the segment's words plus up to 3 words
                                            // before them (copies start 16-byte aligned)
@@ -618,6 +619,13 @@ struct ServerArgs {
     double* part_s;          // [nch][blocks per chunk]: one fp64 partial per block
     uint32_t* status;
     const DpRoute* route;    // data-parallel ranks only: where the server plane goes
+    // Folded worker scales (single GPU, few partials per chunk): instead of reading s, every
+    // block reduces the chunk's worker partials itself, in the order of k_scales<ws_tpr>, and
+    // block 0 of the chunk stores them (s_out, s_lazy). part_w null: s is read.
+    const double* part_w;    // [W][nch][nseg]
+    int ws_tpr;              // 1 or 32: threads per row, as launch_scales would pick
+    float* s_out;            // [W][nch]
+    float* s_lazy;           // [W][nch]
 };
 
 // Pipeline depth of k_server: two stages while they fit next to the tables and a block has
@@ -626,23 +634,69 @@ __host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
     return (W <= 128 && nseg_s > 1) ? 2 : 1;
 }
 
+// Lookup tables. The 4-byte tables (int32 group sums, or the fp32 y table for W <= 8) are read
+// at random entries by all 32 lanes of a warp at once; with one copy of a table several lanes
+// land on the same shared-memory bank (about 3 wavefronts per lookup instead of 1).
+//
+// Bank-private tables cut that for 2, 4 or 8 groups (9 <= W <= 64): every bank holds a whole
+// copy of one group's table. Entry i of the tables is row i of RW = NG * K words (NG groups, K
+// copies each); word g * K + h of a row is copy h of group g's entry. In lookup slot s, lane l
+// reads group (s + l) mod NG from copy (l / NG) mod K. With 4 or 8 groups K = 32 / NG and the
+// lanes that read one group at once use K different banks: one wavefront per lookup (32 KB).
+// With 2 groups K = 8 (16 KB, rows of 16 words): lanes l and l + 16 share a copy and meet in a
+// bank when their entries have the same parity, so a lookup takes 2 wavefronts.
+//
+// The copies cost shared memory (fewer blocks per SM) and a longer table set-up, which pays
+// where a block streams many segments and, for 2 groups (3 blocks per SM instead of 4), where
+// the grid is long enough that its last wave matters little. Otherwise (W <= 8, W > 64, short
+// chunks, small grids) each group's table is one 1 KB copy (measured both ways). Partial
+// replication with lane l reading copy l mod R does not help for R < 16: the cost of a warp's
+// lookup is the busiest bank's load, and with R = 2, 4 or 8 that load stays at about 3.
+__host__ __device__ constexpr int server_copies(int ng) { return ng == 2 ? 8 : 32 / ng; }
+__host__ __device__ inline bool server_bank_private(int W, int64_t nseg_s, int64_t nch) {
+    const int ngroups = (W + 7) / 8;
+    if (nseg_s < 8) return false;
+    if (ngroups == 4 || ngroups == 8) return true;
+    return ngroups == 2 && nch * ((nseg_s + 7) / 8) >= 2048;
+}
+
+// Server segments per block: 16 with bank-private tables for 4 or 8 groups and long chunks
+// (their set-up is spread over more segments), else 8.
+__host__ __device__ inline int server_segs_per_block(int W, int64_t nseg_s, int64_t nch) {
+    return (server_bank_private(W, nseg_s, nch) && (W + 7) / 8 >= 4 && nseg_s >= 16) ? 16 : 8;
+}
+
 // Residuals staged by TMA next to the sign words (STAGE_RES) while the stages stay small enough
-// for several blocks per SM; for wider W they are read into registers instead (measured).
-__host__ __device__ inline bool server_stage_residuals(int W) { return W <= 32; }
+// for several blocks per SM (W <= 32, single-copy tables or the 16 KB tables of 2 groups);
+// otherwise they are read into registers at the top of each segment (measured).
+__host__ __device__ inline bool server_stage_residuals(int W, bool bank_private) {
+    return W <= 32 && (!bank_private || (W + 7) / 8 == 2);
+}
+
+// Bytes of the table region: the bank-private int32 tables or, in the same place, the fp64
+// tables of kModeF64 (one copy of [ngroups][256]); with single-copy tables, the fp64 tables and
+// the int32 tables in the same place, then the y table (W <= 8).
+__host__ __device__ inline size_t server_table_bytes(int W, bool bank_private) {
+    const int ngroups = (W + 7) / 8;
+    const size_t f64 = (size_t)ngroups * 256 * sizeof(double);
+    if (!bank_private) return f64 + 256 * sizeof(float);
+    const size_t tab = (size_t)256 * ngroups * server_copies(ngroups) * sizeof(int32_t);
+    return f64 > tab ? f64 : tab;
+}
 
 // Words of one pipeline stage: wpad plane rows, then the segment's residuals when staged.
 __host__ __device__ inline size_t server_stage_words(int W, bool stage_res) {
     return (size_t)((W + 7) & ~7) * kTileRow + (stage_res ? kSegS : 0);
 }
 
-// Dynamic shared memory of k_server for W workers and `nst` stages (bytes).
-__host__ __device__ inline size_t server_smem_bytes(int W, int nst) {
+// Dynamic shared memory of k_server for W workers, `nst` stages and the table layout (bytes).
+__host__ __device__ inline size_t server_smem_bytes(int W, int nst, bool bank_private) {
     const int wpad = (W + 7) & ~7;
     return 64                                                   // mbarriers, mode, unit
-         + (size_t)nst * server_stage_words(W, server_stage_residuals(W)) * sizeof(uint32_t)
+         + (size_t)nst * server_stage_words(W, server_stage_residuals(W, bank_private)) *
+               sizeof(uint32_t)
          + (size_t)wpad * sizeof(double)                        // scales
-         + (size_t)(wpad / 8) * 256 * sizeof(double)            // per-group tables
-         + 256 * sizeof(float)                                  // y table (W <= 8)
+         + server_table_bytes(W, bank_private)                  // tables
          + kWarps * sizeof(double);                             // reduction
 }
 
@@ -693,19 +747,21 @@ __device__ __forceinline__ void server_issue(const ServerArgs& a, uint32_t* stag
 // the receive planes of all W workers, bits_s points at this rank's first chunk in its own copy
 // of the server plane, and each block then stores its server words into every other rank's copy
 // (the broadcast half of the compressed allreduce, to peer memory).
-template <bool POW2, bool STAGE_RES, bool BCAST = false>
-__global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
+template <bool POW2, bool STAGE_RES, bool BCAST = false, int NG = 0>
+__global__ void __launch_bounds__(kThreads, NG == 8 ? 2 : (NG == 4 || NG == 2 ? 3 : 4))
+k_server(const ServerArgs a) {
     extern __shared__ __align__(16) unsigned char smem_srv[];
     const int W = a.geo.W;
-    const int64_t nsb = (a.geo.nseg_s + kSrvSegsPerBlock - 1) / kSrvSegsPerBlock;
+    const int spb = a.geo.spb;
+    const int64_t nsb = (a.geo.nseg_s + spb - 1) / spb;
     const int64_t k = (int64_t)blockIdx.x / nsb;
     const int64_t b = (int64_t)blockIdx.x - k * nsb;
     const int64_t c0 = k * a.geo.C;
     const int64_t clen = min(a.geo.C, a.geo.d - c0);
     const int64_t nseg_k = (clen + kSegS - 1) / kSegS;
-    const int64_t j0 = b * kSrvSegsPerBlock;
+    const int64_t j0 = b * spb;
     if (j0 >= nseg_k) return;
-    const int nseg_blk = (int)min((int64_t)kSrvSegsPerBlock, nseg_k - j0);
+    const int nseg_blk = (int)min((int64_t)spb, nseg_k - j0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int wpad = (W + 7) & ~7, ngroups = wpad / 8;
     const int nst = server_stages(W, a.geo.nseg_s);
@@ -719,10 +775,15 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     const size_t stage_words = server_stage_words(W, STAGE_RES);
     uint32_t* stages = reinterpret_cast<uint32_t*>(smem_srv + 64);
     double* sw = reinterpret_cast<double*>(stages + (size_t)nst * stage_words);
-    double* lut = sw + wpad;                                  // fp64 tables [ngroups][256]
-    int32_t* ilut = reinterpret_cast<int32_t*>(lut);          // or int32 tables, same place
+    // one table region: the fp64 tables [ngroups][256] (kModeF64), and in the same place the
+    // int32 tables (kModeInt): with NG > 0 bank-private, [256 rows][32 banks], else
+    // [ngroups][256]; without NG the y table (kModeY) follows the fp64 tables
+    constexpr bool BP = NG > 0;
+    double* lut = sw + wpad;
+    int32_t* ilut = reinterpret_cast<int32_t*>(lut);
     float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
-    double* red = reinterpret_cast<double*>(ylut + 256);
+    double* red = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(lut) +
+                                            server_table_bytes(W, BP));
     const double dW = (double)W, invW = 1.0 / (double)W;
 
     if (tid == 0) {
@@ -734,8 +795,30 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
             server_issue<STAGE_RES, BCAST>(a, stages + (size_t)t * stage_words, wpad, &bars[t],
                                            c0, clen, j0 + t);
     }
-    for (int w = tid; w < wpad; w += kThreads)
-        sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
+    if (a.part_w == nullptr) {
+        for (int w = tid; w < wpad; w += kThreads)
+            sw[w] = w < W ? (double)a.s[(int64_t)w * a.geo.nch + k] : 0.0;
+    } else if (a.ws_tpr == 1) {
+        for (int w = tid; w < wpad; w += kThreads) {
+            const bool on = w < W;
+            const int64_t r = (int64_t)w * a.geo.nch + k;
+            const float sv = row_scale<1>(a.part_w, r, on, a.geo.nch, a.geo.nseg, kSeg, a.geo.C,
+                                          a.geo.d, nullptr);
+            sw[w] = on ? (double)sv : 0.0;
+            if (on && b == 0) { a.s_out[r] = sv; a.s_lazy[r] = sv; }
+        }
+    } else {
+        for (int w = warp; w < wpad; w += kWarps) {
+            const bool on = w < W;
+            const int64_t r = (int64_t)w * a.geo.nch + k;
+            const float sv = row_scale<32>(a.part_w, r, on, a.geo.nch, a.geo.nseg, kSeg, a.geo.C,
+                                           a.geo.d, nullptr);
+            if (lane == 0) {
+                sw[w] = on ? (double)sv : 0.0;
+                if (on && b == 0) { a.s_out[r] = sv; a.s_lazy[r] = sv; }
+            }
+        }
+    }
     if constexpr (BCAST)
         for (int st = 0; st < nst; ++st)
             for (int e = W * kTileRow + tid; e < wpad * kTileRow; e += kThreads)
@@ -803,8 +886,7 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
     if (mode == kModeInt) {
         // +-s_w as exact integers in units of u = 2^(emin - 150)
         const int emin = *emin_p;
-        for (int e = tid; e < ngroups * 256; e += kThreads) {
-            const int g = e >> 8, idx = e & 255;
+        auto entry = [&](int g, int idx) {
             int32_t acc = 0;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -814,9 +896,36 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 const int32_t M = bits == 0u ? 0 : (int32_t)(mant << (max(eb, 1) - emin));
                 acc += ((idx >> i) & 1) ? M : -M;
             }
-            ilut[e] = acc;
+            return acc;
+        };
+        if constexpr (BP) {
+            // entry e: group e mod NG (= lane mod NG), index e / NG. Its K copies go to banks
+            // g * K + (q + h) mod K at step q, h = lane / NG: a warp's 32 lanes hold NG groups
+            // x K consecutive entries, so at every step they store to 32 different banks.
+            constexpr int K = server_copies(NG), RW = NG * K;
+            const int h = (lane / NG) % K;
+            for (int e = tid; e < NG * 256; e += kThreads) {
+                const int g = e % NG, idx = e / NG;
+                const int32_t v = entry(g, idx);
+                int32_t* row = ilut + idx * RW + g * K;
+#pragma unroll
+                for (int q = 0; q < K; ++q) row[(q + h) % K] = v;
+            }
+        } else {
+            for (int e = tid; e < ngroups * 256; e += kThreads) ilut[e] = entry(e >> 8, e & 255);
         }
-    } else if (mode != kModeSeq) {
+    } else if (mode == kModeY) {
+        // one group: y itself, from the in-order fp64 sum over the 8 (padded) workers
+        for (int idx = tid; idx < 256; idx += kThreads) {
+            double acc = 0.0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const double sv = sw[i];
+                acc = __dadd_rn(acc, ((idx >> i) & 1) ? sv : -sv);
+            }
+            ylut[idx] = server_average<POW2>(acc, dW, invW);
+        }
+    } else if (mode == kModeF64) {
         // fp64 tables: entry idx of group g = sum over i of (bit i of idx ? s : -s), in order
         for (int e = tid; e < ngroups * 256; e += kThreads) {
             const int g = e >> 8, idx = e & 255;
@@ -827,7 +936,6 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                 acc = __dadd_rn(acc, ((idx >> i) & 1) ? sv : -sv);
             }
             lut[e] = acc;
-            if (g == 0) ylut[idx] = server_average<POW2>(acc, dW, invW);
         }
     }
     __syncthreads();
@@ -899,13 +1007,28 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
                     int32_t acc[kSrvVec];
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c) acc[c] = 0;
-#pragma unroll 2
-                    for (int g = 0; g < ngroups; ++g) {
-                        uint32_t lo, hi;
-                        pattern(g, lo, hi);
-                        const int32_t* L = ilut + g * 256;
+                    if constexpr (BP) {
+                        // slot sl: this lane's group (sl + lane) mod NG, from its own copy
+                        // (integer sums: the order of the groups does not matter)
 #pragma unroll
-                        for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
+                        for (int sl = 0; sl < NG; ++sl) {
+                            const int gs = (sl + lane) % NG;
+                            uint32_t lo, hi;
+                            pattern(gs, lo, hi);
+                            constexpr int K = server_copies(NG), RW = NG * K;
+                            const int32_t* L = ilut + gs * K + (lane / NG) % K;
+#pragma unroll
+                            for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c) * RW];
+                        }
+                    } else {
+#pragma unroll 2
+                        for (int g = 0; g < ngroups; ++g) {
+                            uint32_t lo, hi;
+                            pattern(g, lo, hi);
+                            const int32_t* L = ilut + g * 256;
+#pragma unroll
+                            for (int c = 0; c < kSrvVec; ++c) acc[c] += L[byte_of(lo, hi, c)];
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < kSrvVec; ++c)
@@ -1005,8 +1128,8 @@ __global__ void __launch_bounds__(kThreads) k_server(const ServerArgs a) {
         // (the block's element range is recomputed from k and b, so that nothing else has to
         // stay live through the main loop)
         const DpRoute* rt = a.route;
-        const int64_t e_lo = k * a.geo.C + b * (kSrvSegsPerBlock * kSegS);
-        const int64_t e_hi = min(min((k + 1) * a.geo.C, a.geo.d), e_lo + kSrvSegsPerBlock * kSegS);
+        const int64_t e_lo = k * a.geo.C + b * ((int64_t)spb * kSegS);
+        const int64_t e_hi = min(min((k + 1) * a.geo.C, a.geo.d), e_lo + (int64_t)spb * kSegS);
         const int64_t w_lo = e_lo >> 5, w_hi = (e_hi + 31) >> 5;
         const int64_t gw0 = (rt->kb[rt->rank] * a.geo.C) >> 5;
         for (int p = 0; p < rt->R; ++p) {
@@ -1032,13 +1155,36 @@ struct ApplyArgs {
     const float* S;          // [nch]
     const float* v;          // [ld]
     float* x;                // [d] caller-owned
+    // Folded server scale (at most 8 server partials per chunk): every block sums the chunk's
+    // partials itself in the order of k_scales<1>, and segment 0's block stores S_out, S_lazy.
+    // part_s null: S is read.
+    const double* part_s;    // [nch][nsb]
+    int64_t nsb;             // server blocks per chunk
+    float* S_out;            // [nch]
+    float* S_lazy;           // [nch]
 };
 
-__global__ void __launch_bounds__(kThreads) k_apply(const ApplyArgs a) {
+__global__ void __launch_bounds__(kThreads, 8) k_apply(const ApplyArgs a) {
     int64_t k, j, base, len;
     if (!block_segment<kSeg>(a.geo, a.geo.nseg, k, j, base, len)) return;
     const int tid = threadIdx.x, lane = tid & 31;
-    const float S = a.S[k];
+    float S;
+    if (a.part_s == nullptr) {
+        S = a.S[k];
+    } else {
+        __shared__ float S_sh;
+        if (tid == 0) {
+            // the partial length as a constant (spb is 8 or 16): no 64-bit division
+            S_sh = a.geo.spb == 16
+                ? row_scale<1>(a.part_s, k, true, a.geo.nch, a.nsb, kSegS * 16, a.geo.C, a.geo.d,
+                               nullptr)
+                : row_scale<1>(a.part_s, k, true, a.geo.nch, a.nsb, kSegS * 8, a.geo.C, a.geo.d,
+                               nullptr);
+            if (j == 0) { a.S_out[k] = S_sh; a.S_lazy[k] = S_sh; }
+        }
+        __syncthreads();
+        S = S_sh;
+    }
     const int sh = 4 * (lane & 7);
 #pragma unroll
     for (int it = 0; it < kItems; ++it) {

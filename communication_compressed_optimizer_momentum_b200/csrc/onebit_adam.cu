@@ -1,7 +1,8 @@
 // onebit_adam.cu -- host side of the C ABI declared in include/onebit_adam.h: argument checks,
 // the workspace layout, the launch sequence of one step and the state/timing helpers.
 //
-// One compressed step is five launches on the caller's stream, ordered by the stream alone
+// One compressed step is five launches on the caller's stream (three for small buckets, whose
+// chunk-scale reductions fold into the server and apply kernels), ordered by the stream alone
 // (no kernel waits on another, so nothing can spin or hang):
 //   k_worker  -> k_scales (worker)  -> k_server -> k_scales (server) -> k_apply
 // The boundary between k_worker/k_scales and k_server is where the compressed allreduce of the
@@ -222,22 +223,52 @@ bool is_dp(const onebit_adam_s* h) { return h->dp.R > 0; }
 
 int64_t step_blocks(const Geometry& g) { return g.nch * g.nseg; }
 int64_t server_blocks_per_chunk(const Geometry& g) {
-    return ceil_div(g.nseg_s, kSrvSegsPerBlock);
+    return ceil_div(g.nseg_s, g.spb);
 }
 int64_t server_blocks(const Geometry& g) { return g.nch * server_blocks_per_chunk(g); }
 
-// The k_server instantiation for W workers: exact scaling for power-of-two W, residuals staged
-// by TMA for narrow W.
+// Small chunk-scale reductions are folded into the kernel that consumes them (one launch less
+// each, which is what small buckets pay for): the worker scales into the server kernel's
+// prologue when a chunk has at most 8 server blocks and few partials (each of those blocks
+// reduces them itself, in the order of the separate reduction), the server scale into the
+// apply kernel when a chunk has at most 8 server partials.
+bool fold_worker_scales(const Geometry& g) {
+    return server_blocks_per_chunk(g) <= 8 && g.nseg <= 1024 && (int64_t)g.W * g.nseg <= 8192;
+}
+bool fold_server_scales(const Geometry& g) { return server_blocks_per_chunk(g) <= 8; }
+int launches_per_step(const Geometry& g) {
+    return kLaunchesPerStep - (fold_worker_scales(g) ? 1 : 0) - (fold_server_scales(g) ? 1 : 0);
+}
+
+// The k_server instantiation for a geometry: exact scaling for power-of-two W; bank-private
+// int32 tables (unrolled over the 4 or 8 groups) where server_bank_private picks them, else
+// single-copy tables with the residuals staged by TMA for W <= 32.
 using ServerKernel = void (*)(ServerArgs);
-ServerKernel server_kernel(int W) {
-    const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W);
-    if (pow2) return staged ? k_server<true, true> : k_server<true, false>;
-    return staged ? k_server<false, true> : k_server<false, false>;
+template <bool POW2>
+ServerKernel server_kernel_pow2(const Geometry& g) {
+    const bool bp = server_bank_private(g.W, g.nseg_s, g.nch);
+    if (bp) {
+        const int ngroups = (g.W + 7) / 8;
+        if (ngroups == 2)
+            return server_stage_residuals(g.W, true) ? k_server<POW2, true, false, 2>
+                                                     : k_server<POW2, false, false, 2>;
+        return ngroups == 4 ? k_server<POW2, false, false, 4> : k_server<POW2, false, false, 8>;
+    }
+    return server_stage_residuals(g.W, false) ? k_server<POW2, true> : k_server<POW2, false>;
+}
+ServerKernel server_kernel(const Geometry& g) {
+    return (g.W & (g.W - 1)) == 0 ? server_kernel_pow2<true>(g) : server_kernel_pow2<false>(g);
+}
+
+// Dynamic shared memory of the single-GPU server kernel of a geometry.
+size_t server_smem(const Geometry& g) {
+    return server_smem_bytes(g.W, server_stages(g.W, g.nseg_s),
+                             server_bank_private(g.W, g.nseg_s, g.nch));
 }
 
 // The same for a data-parallel rank: the server plane is broadcast to every rank.
 ServerKernel server_kernel_dp(int W) {
-    const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W);
+    const bool pow2 = (W & (W - 1)) == 0, staged = server_stage_residuals(W, false);
     if (pow2) return staged ? k_server<true, true, true> : k_server<true, false, true>;
     return staged ? k_server<false, true, true> : k_server<false, false, true>;
 }
@@ -492,13 +523,13 @@ int dp_compressed_phase(onebit_adam_s* h, int phase, float* x, const void* grads
             const float* rs = reinterpret_cast<const float*>(dp.xch + dp.xl.rscales);
             ServerArgs sa{gs, nullptr, planes, rs, h->es, h->S_lazy, h->bits_s + dp.e0 / 32,
                           h->part_s, h->status, dp.route_dev};
-            const size_t ssm = server_smem_bytes(gs.W, server_stages(gs.W, gs.nseg_s));
+            const size_t ssm = server_smem_bytes(gs.W, server_stages(gs.W, gs.nseg_s), false);
             server_kernel_dp(gs.W)<<<(unsigned)server_blocks(gs), kThreads, ssm, st>>>(sa);
             ONEBIT_CUDA(cudaGetLastError());
         }
         record(h, 3, st);
         rc = launch_scales_dp<true>(gs.nch, gs.C, gs.d, h->part_s, gs.nch,
-                                    server_blocks_per_chunk(gs), kSegS * kSrvSegsPerBlock,
+                                    server_blocks_per_chunk(gs), kSegS * gs.spb,
                                     nullptr, h->S_lazy, dp.route_dev, st);
     } else {
         record(h, 4, st);
@@ -556,6 +587,7 @@ int onebit_adam_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float 
     g.nch = ceil_div(d, C);
     g.nseg = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSeg);
     g.nseg_s = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSegS);
+    g.spb = server_segs_per_block(W, g.nseg_s, g.nch);
     g.ld = round_up(d > 0 ? d : 1, 64);
     h->nw = ceil_div(d, 32);
     g.ldw = round_up(h->nw > 0 ? h->nw : 1, 4);
@@ -623,13 +655,13 @@ int onebit_adam_bind(onebit_adam_t h, void* workspace, uint64_t bytes, int32_t g
         dp.connected = false;
         dp.next_phase = 0;
         dp.phase_kind = 0;
-        const int ssm = (int)server_smem_bytes(dp.Wg, server_stages(dp.Wg, dp.gs.nseg_s));
+        const int ssm = (int)server_smem_bytes(dp.Wg, server_stages(dp.Wg, dp.gs.nseg_s), false);
         ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel_dp(dp.Wg),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
         ONEBIT_CUDA(cudaMemsetAsync(dp.xch, 0, dp.xl.total, st));
     } else {
-        const int ssm = (int)server_smem_bytes(h->geo.W, server_stages(h->geo.W, h->geo.nseg_s));
-        ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel(h->geo.W),
+        const int ssm = (int)server_smem(h->geo);
+        ONEBIT_CUDA(cudaFuncSetAttribute(server_kernel(h->geo),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, ssm));
     }
     // m and v start at zero (Adam); the rest is cleared too so padding is deterministic.
@@ -747,21 +779,29 @@ int onebit_adam_compressed_step(onebit_adam_t h, float* x, const void* grads, fl
                                  : launch_worker<float>(h, grads, st);
     if (rc != ONEBIT_OK) return rc;
     record(h, 1, st);
-    rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out, h->s_lazy, st);
-    if (rc != ONEBIT_OK) return rc;
+    const bool fold_ws = fold_worker_scales(g), fold_ss = fold_server_scales(g);
+    if (!fold_ws) {
+        rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out, h->s_lazy,
+                           st);
+        if (rc != ONEBIT_OK) return rc;
+    }
     record(h, 2, st);
     ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s, h->part_s,
-                  h->status};
-    const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
+                  h->status, nullptr, fold_ws ? h->part_w : nullptr, g.nseg <= 8 ? 1 : 32,
+                  h->s_out, h->s_lazy};
+    const size_t ssm = server_smem(g);
     const unsigned sblocks = (unsigned)server_blocks(g);
-    server_kernel(g.W)<<<sblocks, kThreads, ssm, st>>>(sa);
+    server_kernel(g)<<<sblocks, kThreads, ssm, st>>>(sa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 3, st);
-    rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
-                       kSegS * kSrvSegsPerBlock, h->S_out, h->S_lazy, st);
-    if (rc != ONEBIT_OK) return rc;
+    if (!fold_ss) {
+        rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
+                           kSegS * g.spb, h->S_out, h->S_lazy, st);
+        if (rc != ONEBIT_OK) return rc;
+    }
     record(h, 4, st);
-    ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, x};
+    ApplyArgs pa{g, h->eps, lr, h->bits_s, h->S_out, h->v, x,
+                 fold_ss ? h->part_s : nullptr, server_blocks_per_chunk(g), h->S_out, h->S_lazy};
     k_apply<<<blocks, kThreads, 0, st>>>(pa);
     ONEBIT_CUDA(cudaGetLastError());
     record(h, 5, st);
@@ -969,7 +1009,7 @@ int onebit_adam_info(onebit_adam_t h, int64_t out[8]) {
     out[4] = h->phase;
     out[5] = h->steps;
     out[6] = h->gtype;
-    out[7] = is_dp(h) ? kLaunchesPerStepDp : kLaunchesPerStep;
+    out[7] = is_dp(h) ? kLaunchesPerStepDp : launches_per_step(h->geo);
     return ONEBIT_OK;
 }
 
@@ -1057,6 +1097,7 @@ int onebit_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float be
     gs.nch = dp.kb[rank + 1] - dp.kb[rank];
     gs.nseg = g.nseg;      // the global segment counts: block partials and their reduction
     gs.nseg_s = g.nseg_s;  // order are those of the single-GPU step
+    gs.spb = g.spb;
     gs.ld = round_up(std::max<int64_t>(gs.d, 1), 64);
     gs.ldw = dp_ldw(*h, rank);
     gs.W = W;
@@ -1372,14 +1413,14 @@ int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* 
         if (sync) {
             ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s,
                           h->part_s, h->status};
-            const size_t ssm = server_smem_bytes(g.W, server_stages(g.W, g.nseg_s));
-            server_kernel(g.W)<<<(unsigned)server_blocks(g), kThreads, ssm, st>>>(sa);
+            const size_t ssm = server_smem(g);
+            server_kernel(g)<<<(unsigned)server_blocks(g), kThreads, ssm, st>>>(sa);
             ONEBIT_CUDA(cudaGetLastError());
         }
         record(h, 3, st);
         if (sync) {
             rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
-                               kSegS * kSrvSegsPerBlock, h->S_out, h->S_lazy, st);
+                               kSegS * g.spb, h->S_out, h->S_lazy, st);
             if (rc != ONEBIT_OK) return rc;
         }
         record(h, 4, st);
@@ -1558,6 +1599,7 @@ extern "C" int onebit_compress_static(const float* x, int64_t n, int64_t C, uint
     g.nch = nch;
     g.nseg = nseg;
     g.W = 1;
+    g.spb = 8;
     // every slot read by the reduction was written by k_compress_partials in this same call,
     // so nothing in the shared array has to be cleared first
     return launch_scales(g, part, nch, nseg, kSeg, scales, scales, st);

@@ -65,7 +65,9 @@ typedef enum {
     ONEBIT_STATE_ES = 3,    /* server residual e_s, fp32[d]                          (get/set) */
     ONEBIT_STATE_SW = 4,    /* last step's worker scales s, fp32[W][nch]             (get) */
     ONEBIT_STATE_SS = 5,    /* last step's server scales S, fp32[nch]                (get) */
-    ONEBIT_STATE_BITSW = 6, /* last step's worker sign planes, uint32[W][ceil(d/32)] (get) */
+    ONEBIT_STATE_BITSW = 6, /* last step's worker sign planes, uint32[W][ceil(d/32)] (get;
+                               rebuilt from the stored x_w: on one GPU the workers' signs are
+                               kept grouped by 8 workers, one byte per element) */
     ONEBIT_STATE_BITSS = 7  /* last step's server sign plane, uint32[ceil(d/32)]     (get) */
 } onebit_state;
 
@@ -196,7 +198,8 @@ int onebit_adam_status(onebit_adam_t h, void* stream, uint32_t* flags);
 /*
  * Shape and progress: out[0..7] = d, W, C, number of chunks, phase (0 unbound, 1 warm-up,
  * 2 compressed), compressed steps taken, gradient dtype (-1 unbound), kernel launches per
- * compressed step.
+ * compressed step (5; 3 or 4 for small buckets, whose chunk-scale reductions fold into the
+ * server and apply kernels; 7 for a data-parallel rank).
  */
 int onebit_adam_info(onebit_adam_t h, int64_t out[8]);
 
@@ -205,8 +208,9 @@ int onebit_adam_info(onebit_adam_t h, int64_t out[8]);
  * recording the next max_steps compressed steps (later steps are not recorded); 0 stops and
  * frees the events. onebit_adam_timing_read waits for the last recorded event and returns, in
  * ms_out[0..4], the summed device time of the worker kernel, the worker-scale reduction, the
- * server kernel, the server-scale reduction and the apply kernel, and the number of recorded
- * steps in *steps; it then starts a new recording window of the same length.
+ * server kernel, the server-scale reduction and the apply kernel (a reduction folded into the
+ * next kernel reads 0), and the number of recorded steps in *steps; it then starts a new
+ * recording window of the same length.
  */
 int onebit_adam_timing(onebit_adam_t h, int32_t max_steps);
 int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps);

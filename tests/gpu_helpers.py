@@ -257,4 +257,18 @@ def run_parity(wl: wls.Workload, chunks: Optional[List[int]] = None,
     del g, x, opt
     torch.cuda.empty_cache()
     log("parity %s: %s" % (wl.name, stats))
+    record_stats(wl.name, stats)
     return stats
+
+
+def record_stats(name: str, stats: dict) -> None:
+    """Append one run's parity counts to the JSON-lines file named by ONEBIT_PARITY_LOG (if
+    set), so that a whole test session's exact-match totals can be read afterwards."""
+    import json
+    import os
+    path = os.environ.get("ONEBIT_PARITY_LOG")
+    if not path:
+        return
+    keep = {k: v for k, v in stats.items() if isinstance(v, (int, float))}
+    with open(path, "a") as f:
+        f.write(json.dumps(dict(keep, workload=name)) + "\n")

@@ -21,7 +21,8 @@ import torch
 import communication_compressed_optimizer_momentum_b200 as ob
 import oracle
 from communication_compressed_optimizer_momentum_b200 import workloads as wls
-from gpu_helpers import DEV, RTOL, TIE, expand, padding_is_zero, rel_x, to_np, unpack_bits
+from gpu_helpers import (DEV, RTOL, TIE, expand, padding_is_zero, record_stats, rel_x, to_np,
+                         unpack_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -159,6 +160,7 @@ def _run(wl, H, K, steps, chunks=None, lr_scale=1.0):
     torch.cuda.empty_cache()
     assert flags == 0, flags
     print("0/1 parity %s H=%d K=%d: %s" % (wl.name, H, K, stats))
+    record_stats("zero_one_%s_H%d_K%d" % (wl.name, H, K), stats)
     return stats
 
 
@@ -240,3 +242,27 @@ def test_zero_one_rejects_the_onebit_step_and_vice_versa():
         ob.onebit01_step(a.h, x, g, 1e-3)
     assert e.value.code == -3
     a.close()
+
+
+def test_bench_zero_one_line():
+    """bench.py --variant zero_one prints one JSON line: every step counted (local and
+    synchronising), one launch per local step and five per synchronising step, the roofline over
+    the interval's average bytes."""
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--workload", "smoke_1m",
+                        "--variant", "zero_one", "--sync-every", "3", "--refresh-every", "1",
+                        "--steps", "6", "--warmup", "3", "--no-e2e", "--no-cpu-baseline"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["config"]["variant"] == "0/1 Adam" and j["config"]["sync_every"] == 3
+    assert j["gpu_launches"] == 6 + 4 * 2
+    assert j["value"] > 0 and j["status_flags"] == 0
+    roof = j["roofline"]
+    assert roof["bound"] == "hbm" and abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9

@@ -90,6 +90,40 @@ def test_ncu_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
     assert bench.ncu_traffic("bert_large_bucket") == {}
 
 
+def test_traffic_summary_is_written_from_an_ncu_csv(tmp_path, monkeypatch):
+    hdr = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream",'
+           '"Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit",'
+           '"Metric Value"')
+    names = {"worker": "void k_worker<unsigned short, 1, 1, 8, 0>(WorkerArgs)",
+             "server": "void k_server<1, 1, 0>(ServerArgs)", "apply": "k_apply(ApplyArgs)"}
+    lines = ["==PROF== Connected to process 1", hdr]
+    figures = {}
+    for i, (launch, k) in enumerate([(0, "worker"), (0, "server"), (0, "apply"),
+                                     (1, "worker"), (1, "server"), (1, "apply")]):
+        rd, wr, ns = 1000 * (i + 1), 500 * (i + 1), 10 * (i + 1)
+        figures[k] = (rd, wr, ns)      # the later launch of each kernel is the one kept
+        for m, v in (("dram__bytes_read.sum", rd), ("dram__bytes_write.sum", wr),
+                     ("gpu__time_duration.sum", ns)):
+            lines.append('"%d","1","p","h","%s","1","7","(256, 1, 1)","(8, 1, 1)","0","10.0",'
+                         '"Command line profiler metrics","%s","byte","%s"'
+                         % (i, names[k], m, format(v, ",")))
+    csv_path = tmp_path / "t.csv"
+    csv_path.write_text("\n".join(lines) + "\n")
+    out = tmp_path / "traffic.json"
+    cap = 1 << 20
+    j = bench.write_traffic_json(str(csv_path), "bert_large_bucket", cap, "cmd", out=str(out))
+    wl = wls.WORKLOADS["bert_large_bucket"]
+    kb = wl.kernel_bytes_per_param()
+    for k, (rd, wr, ns) in figures.items():
+        got = j["kernels"][k]
+        assert (got["dram_bytes_read"], got["dram_bytes_write"], got["duration_ns"]) == (rd, wr, ns)
+        assert got["dram_over_algorithmic"] == round((rd + wr) / (kb[k] * cap), 4)
+        assert got["dram_bytes_per_launch_full"] == round((rd + wr) * wl.d / cap)
+    monkeypatch.setattr(bench, "TRAFFIC_JSON", str(out))
+    assert bench.ncu_traffic("bert_large_bucket") == {
+        k: float(round((rd + wr) * wl.d / cap)) for k, (rd, wr, _) in figures.items()}
+
+
 def test_committed_traffic_summary_parses():
     if not os.path.exists(bench.TRAFFIC_JSON):
         pytest.skip("no ncu traffic summary committed for the current kernels")
