@@ -11,7 +11,9 @@
 // the interval's learning rates) becomes every worker's momentum, and u_w restarts at zero.
 // Neither is written: the next step rebuilds mbar = +-fl(S_k / Gamma) from the server plane
 // and takes u_w = 0 (kZoMBar), as the first step after the freeze takes the warm-up momentum
-// (kZoMShared); only the steps in between read and write the per-worker buffers (kZoMWorker).
+// (kZoMShared). That first step of an interval stores m_w only: its u_w = fl(0 + fl(lr * m_w))
+// is rebuilt from the stored m_w by the next step and by the exports, with the same two
+// roundings (kZoMWorkerU1). The steps after it read and write both buffers (kZoMWorker).
 #pragma once
 
 #include "kernels.cuh"
@@ -24,6 +26,8 @@ enum ZoSource : int {
                      // u_w = 0
     kZoMBar = 1,     // mbar = +-fl(S_k / Gamma) by the last synchronisation's server plane; u_w = 0
     kZoMWorker = 2,  // each worker's own m_w and u_w (steps after a local step)
+    kZoMWorkerU1 = 3,  // each worker's own m_w; u_w = fl(0 + fl(lr_first * m_w)), not stored
+                       // (the step after the interval's first step)
 };
 
 struct ZoArgs {
@@ -34,6 +38,7 @@ struct ZoArgs {
     const uint32_t* bits_s;  // [ldw] last synchronisation's server plane (kZoMBar)
     const float* S;          // [nch] its server scales (kZoMBar)
     float gamma_prev;        // its Gamma (kZoMBar)
+    float lr_first;          // the learning rate of the interval's first step (kZoMWorkerU1)
     float* mw;               // [W][ld] per-worker momentum
     float* uw;               // [W][ld] per-worker accumulated update
     const void* g;           // [W][d] caller-owned, GT
@@ -45,12 +50,16 @@ struct ZoArgs {
 };
 
 // One step of every worker for one segment (a block owns a kSeg segment and loops over the W
-// workers, like k_worker). Local step: m_w = b1 m + (1-b1) g_w; u_w += lr m_w, stored. SYNC
+// workers, like k_worker). Local step: m_w = b1 m + (1-b1) g_w; u_w += lr m_w, stored (u_w only
+// when it did not start at zero: the first step's is rebuilt, kZoMWorkerU1). SYNC
 // (the step that ends with a synchronisation): the same m_w and u_w, then x_w = u_w + e_w
 // compressed as in k_worker (sign bits grouped by 8 workers, lazy residual, fp64 partials of the
 // chunk norm); m_w and u_w are not stored, since the synchronisation replaces them.
+// No blocks-per-SM bound: with the three per-worker streams of a step (and the residual of the
+// synchronising one) the bound of k_worker made the compiler spill, which cost up to 16% of a
+// step (measured); at the registers it picks (32-60) the kernel runs without spills.
 template <typename GT, bool VEC, int EPT, bool SYNC>
-__global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k01_worker(const ZoArgs a) {
+__global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
     constexpr int ITEMS = kSeg / (kThreads * EPT);
     constexpr int LPW = 32 / EPT;  // lanes that share one 32-element word of the server plane
     extern __shared__ double red_w[];  // [W][kWarps] (SYNC)
@@ -123,6 +132,13 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k01_worker(const Z
                         ld4(uwp + off + 4 * h, t4);
 #pragma unroll
                         for (int c = 0; c < 4; ++c) u0[4 * h + c] = t4[c];
+                    } else if (src == kZoMWorkerU1) {
+                        ld4(mwp + off + 4 * h, t4);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            m0[4 * h + c] = t4[c];
+                            u0[4 * h + c] = __fadd_rn(0.0f, __fmul_rn(a.lr_first, t4[c]));
+                        }
                     }
                     if (SYNC) {
                         ld4(ew + off + 4 * h, t4);
@@ -145,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, EPT == 8 ? 6 : 8) k01_worker(const Z
                         const float tm[4] = {mn[4 * h], mn[4 * h + 1], mn[4 * h + 2], mn[4 * h + 3]};
                         const float tu[4] = {un[4 * h], un[4 * h + 1], un[4 * h + 2], un[4 * h + 3]};
                         st4(mwp + off + 4 * h, tm);
-                        st4(uwp + off + 4 * h, tu);
+                        if (src >= kZoMWorker) st4(uwp + off + 4 * h, tu);
                     }
                 }
             } else {
@@ -253,6 +269,9 @@ __global__ void k01_export(const ZoArgs a, int64_t i0, int64_t n, float* mw_out,
         if (a.src == kZoMWorker) {
             m = a.mw[r * a.geo.ld + i];
             u = a.uw[r * a.geo.ld + i];
+        } else if (a.src == kZoMWorkerU1) {
+            m = a.mw[r * a.geo.ld + i];
+            u = __fadd_rn(0.0f, __fmul_rn(a.lr_first, m));
         } else {
             u = 0.0f;
             if (a.src == kZoMShared) {
@@ -267,13 +286,17 @@ __global__ void k01_export(const ZoArgs a, int64_t i0, int64_t n, float* mw_out,
     }
 }
 
-// Worker w's local model, out[i] = x[i] - u_w[i] / (sqrt(v[i]) + eps), for i < d.
-__global__ void k01_local_model(const float* x, const float* uw, int zero_u, const float* v,
-                                float eps, int64_t d, float* out) {
+// Worker w's local model, out[i] = x[i] - u_w[i] / (sqrt(v[i]) + eps), for i < d, with u_w
+// as the state holds it (src as in ZoArgs; mw, uw the worker's rows).
+__global__ void k01_local_model(const float* x, const float* mw, const float* uw, int src,
+                                float lr_first, const float* v, float eps, int64_t d,
+                                float* out) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < d;
          i += (int64_t)gridDim.x * blockDim.x) {
         const float den = __fadd_rn(__fsqrt_rn(v[i]), eps);
-        const float u = zero_u ? 0.0f : uw[i];
+        const float u = src == kZoMWorker     ? uw[i]
+                        : src == kZoMWorkerU1 ? __fadd_rn(0.0f, __fmul_rn(lr_first, mw[i]))
+                                              : 0.0f;
         out[i] = __fsub_rn(x[i], __fdiv_rn(u, den));
     }
 }

@@ -103,6 +103,7 @@ struct ZoState {
     int64_t syncs = 0;
     float gamma = 0.0f;        // fp32 sum of the learning rates since the last synchronisation
     float gamma_prev = 0.0f;   // Gamma of the last synchronisation (mbar = ubar / gamma_prev)
+    float lr_first = 0.0f;     // learning rate of the interval's first step (kZoMWorkerU1)
     int src = kZoMShared;      // where the next step's momentum comes from (ZoSource)
 };
 
@@ -1340,6 +1341,7 @@ ZoArgs zo_args(onebit_adam_s* h, const void* grads, float lr) {
     a.bits_s = h->bits_s;
     a.S = h->S_out;
     a.gamma_prev = h->zo.gamma_prev;
+    a.lr_first = h->zo.lr_first;
     a.mw = h->mw;
     a.uw = h->uw;
     a.g = grads;
@@ -1443,7 +1445,13 @@ int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* 
     } else {
         z.gamma = gamma;
         ++z.t;
-        z.src = kZoMWorker;
+        // the interval's first step stored m_w only; the next one rebuilds its u_w
+        if (z.src == kZoMShared || z.src == kZoMBar) {
+            z.src = kZoMWorkerU1;
+            z.lr_first = lr;
+        } else {
+            z.src = kZoMWorker;
+        }
     }
     return ONEBIT_OK;
 }
@@ -1487,7 +1495,8 @@ int onebit01_local_model(onebit_adam_t h, int32_t w, const float* x, float* out,
     if (g.d == 0) return ONEBIT_OK;
     const unsigned blocks = (unsigned)std::min<int64_t>(ceil_div(g.d, kThreads), 148 * 32);
     k01_local_model<<<blocks, kThreads, 0, as_stream(stream)>>>(
-        x, h->uw + (int64_t)w * g.ld, h->zo.src != kZoMWorker, h->v, h->eps, g.d, out);
+        x, h->mw + (int64_t)w * g.ld, h->uw + (int64_t)w * g.ld, h->zo.src, h->zo.lr_first,
+        h->v, h->eps, g.d, out);
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
 }

@@ -85,21 +85,26 @@ class Workload:
         """The 0/1 Adam variant's minimum HBM bytes per parameter per step, averaged over one
         interval of H steps (a synchronisation every H steps, a variance refresh at every K-th
         one). The first step after a synchronisation rebuilds the shared momentum estimate from
-        the server plane (1/8) and writes every worker's momentum and accumulated update
-        (W*(G + 8)); the steps in between read and write both (W*(G + 16)); the synchronising
-        step reads them, compresses u_w + e_w (residual read and written, sign plane written:
-        W*(G + 16.125)), then the server stage (W/8 + 8.125) and the synchronised step (server
-        plane, v, x: 12.125, plus 4 when v is refreshed). With H = 1 every step is the 1-bit
-        Adam step's bytes."""
+        the server plane (1/8) and writes every worker's momentum (W*(G + 4)); its accumulated
+        update lr * m_w is not stored but rebuilt by the next step, which reads the momentum and
+        writes both (W*(G + 12)); the steps after that read and write both (W*(G + 16)). The
+        synchronising step reads them (only the momentum when it is the interval's second
+        step), compresses u_w + e_w (residual read and written, sign plane written: W*(G +
+        16.125), or W*(G + 12.125)), then the server stage (W/8 + 8.125) and the synchronised
+        step (server plane, v, x: 12.125, plus 4 when v is refreshed). With H = 1 every step is
+        the 1-bit Adam step's bytes."""
         G, W = self.grad_bytes, self.W
         server = W / 8.0 + 8.125
         apply = 12.125 + (4.0 / K if K > 0 else 0.0)
         if H == 1:
             return W * (G + 8.125) + 0.125 + server + apply
-        first = W * (G + 8.0) + 0.125
-        middle = (H - 2) * W * (G + 16.0)
+        first = W * (G + 4.0) + 0.125
+        if H == 2:
+            return (first + W * (G + 12.125) + server + apply) / 2
+        second = W * (G + 12.0)
+        middle = (H - 3) * W * (G + 16.0)
         sync = W * (G + 16.125) + server + apply
-        return (first + middle + sync) / H
+        return (first + second + middle + sync) / H
 
     def kernel_bytes_per_param(self) -> dict:
         """The same minimum, split by the three streaming kernels of the step."""

@@ -450,7 +450,9 @@ int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* 
 /*
  * out[0..5] = H, K, steps since the last synchronisation, synchronisations so far, where the
  * next step's momentum comes from (0: the warm-up momentum, 1: the last synchronisation's
- * mbar, 2: each worker's own), launches of the next step (5 when it synchronises, else 1).
+ * mbar, 2: each worker's own, 3: each worker's own, with the accumulated update of the
+ * interval's first step rebuilt from it rather than stored), launches of the next step (5 when
+ * it synchronises, else 1).
  * Host only; ONEBIT_ERR_ARG for a 1-bit Adam handle.
  */
 int onebit01_info(onebit_adam_t h, int64_t out[6]);
