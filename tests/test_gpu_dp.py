@@ -42,6 +42,10 @@ CASES = {
     "r2_w64": (_wl(F32, 40_000, 64, 4096), 2),                 # residuals not staged (W > 32)
     "r5_w10": (_wl(F32, 60_000, 10, 2048), 5),                  # W not a power of two
     "r3_spread": (_wl(F32, 30_000, 6, 1024, last_worker_sigma=1e-8), 3),  # in-order decode
+    # the single handle's server uses bank-private tables and 16 segments per block; the ranks'
+    # server blocks cover the same 16 segments with one-copy tables
+    "r2_w64_bank_private": (_wl(F32, 300_000, 64, 131_072), 2),
+    "r2_w30_bank_private_bf16": (_wl(BF16, 200_003, 30, 65_536, grad_kind="normal"), 2),
 }
 
 NAMES = ("m", "v", "e_w", "e_s", "s", "S", "bits_w", "bits_s")

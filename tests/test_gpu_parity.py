@@ -46,6 +46,10 @@ SMALL = [
     small(40_000, 16, 8192, beta1=0.0, last_worker_sigma=1e-2),
     small(40_000, 16, 8192, beta1=0.0, last_worker_sigma=1e-10),
     small(40_000, 12, 8192, beta1=0.0, last_worker_sigma=1e-10),
+    # bank-private server tables: 4 groups with W not a power of two (8 segments per block),
+    # 8 groups with a ragged last chunk (16 segments per block)
+    small(150_000, 30, 40_000, "bf16"),
+    small(300_007, 60, 69_984),
 ]
 
 
@@ -59,6 +63,19 @@ def test_compressed_parity_small(wl):
     else:
         assert st["inexact_chunks"] == 0
     assert st["status_flags"] == 0
+
+
+def test_two_group_bank_private_tables_sampled():
+    """The bank-private tables of 2 groups need a grid of at least 2048 server blocks: W = 12
+    (not a power of two) over 2^26 + 4099 parameters in 2^18-element chunks (257 chunks of 8
+    server blocks each), checked on sampled chunks including the ragged last one."""
+    wl = small((1 << 26) + 4099, 12, 1 << 18, "bf16", "outlier_normal", warm=2, comp=3)
+    free, _ = torch.cuda.mem_get_info()
+    if free < 8e9:
+        pytest.skip("needs about 8 GB of free device memory")
+    assert wl.nch * (((wl.C + 4095) // 4096 + 7) // 8) >= 2048
+    st = run_parity(wl, chunks=[0, 1, wl.nch - 1], teacher_steps=(1, 2, 3), free_steps=0)
+    assert st["inexact_chunks"] == 0 and st["status_flags"] == 0
 
 
 def test_smoke_1m_workload():
