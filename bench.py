@@ -270,6 +270,17 @@ def warmup_phase(wl, warm_ms):
             "achieved_gbs": nbytes / (ms / 1e3) / 1e9}
 
 
+def step_distribution(step_ms):
+    """p10 / p50 / p90 of single steps' device times (ms), nearest-rank; None without any."""
+    if not step_ms:
+        return None
+    v = sorted(step_ms)
+
+    def q(p):
+        return v[min(len(v) - 1, max(0, int(round(p * (len(v) - 1)))))]
+    return {"p10": q(0.1), "p50": q(0.5), "p90": q(0.9), "steps": len(v)}
+
+
 def whole_job_rate(units_per_rank, world, ms_max):
     """Units all ranks processed per second, timed by the slowest rank."""
     return units_per_rank * world / (ms_max / 1e3)
@@ -499,6 +510,7 @@ def run_ours(args):
         for _ in range(args.steps):
             opt.step(x, g, wl.lr)
         torch.cuda.synchronize()
+    per_step = opt.timing_steps(args.steps) if graph is None else []
     kernel_ms, nrec = opt.timing_read()
     opt.timing(0)
     time.sleep(0.3)
@@ -581,6 +593,12 @@ def run_ours(args):
             "pct_of_nominal_hbm": 100.0 * achieved_step_gbs / NOMINAL_HBM_GBS,
             "algorithmic_bytes_per_step": step_bytes,
             "kernel_ms_per_step": {k2: v2 / max(nrec, 1) for k2, v2 in kernel_ms.items()},
+            # the distribution of single steps' device time (first to last event of each step,
+            # from the same per-kernel events)
+            "step_ms_distribution": step_distribution(per_step),
+            # one worker's message against its fp32 vector: d/8 sign bytes + one fp32 scale per
+            # chunk, against 4d bytes
+            "compression_ratio": 4.0 * wl.d / (wl.d / 8.0 + 4.0 * wl.nch),
             "roofline": {"bound": "hbm", "kernel": "worker", "achieved": worker_gbs,
                          "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": (worker_gbs / peak) if worker_gbs else None,

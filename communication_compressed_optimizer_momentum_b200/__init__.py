@@ -169,6 +169,17 @@ def onebit_adam_timing_read(h) -> Tuple[dict, int]:
     return dict(zip(KERNELS, list(ms))), n.value
 
 
+def onebit_adam_timing_steps(h, cap: int) -> list:
+    """The device time (ms) of each step of the current recording window, at most cap."""
+    if cap < 0:
+        raise ValueError("cap must be >= 0")
+    ms = (ctypes.c_double * max(cap, 1))()
+    n = ctypes.c_int32()
+    _check(_abi.lib().onebit_adam_timing_steps(_handle(h), ms, cap, ctypes.byref(n)),
+           "onebit_adam_timing_steps")
+    return list(ms)[:min(cap, n.value)]
+
+
 def onebit_adam_destroy(h) -> None:
     _abi.lib().onebit_adam_destroy(_handle(h))
 
@@ -451,6 +462,10 @@ class OneBitAdam:
 
     def timing_read(self):
         return onebit_adam_timing_read(self.h)
+
+    def timing_steps(self, cap: int = 1 << 16):
+        """Device time (ms) of each step recorded in the current window (before timing_read)."""
+        return onebit_adam_timing_steps(self.h, cap)
 
     def close(self) -> None:
         if getattr(self, "h", None) is not None:

@@ -36,6 +36,8 @@ SIGNATURES = {
     "onebit_adam_info": (INT, [P, ctypes.POINTER(I64)]),
     "onebit_adam_timing": (INT, [P, I32]),
     "onebit_adam_timing_read": (INT, [P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(I32)]),
+    "onebit_adam_timing_steps": (INT, [P, ctypes.POINTER(ctypes.c_double), I32,
+                                       ctypes.POINTER(I32)]),
     "onebit_adam_destroy": (None, [P]),
     "onebit_pack": (INT, [P, I64, P, P]),
     "onebit_unpack": (INT, [P, P, I64, I64, P, P]),

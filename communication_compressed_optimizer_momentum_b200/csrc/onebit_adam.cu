@@ -1052,6 +1052,21 @@ int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps) {
     return ONEBIT_OK;
 }
 
+int onebit_adam_timing_steps(onebit_adam_t h, double* step_ms, int32_t cap, int32_t* steps) {
+    if (!valid_handle(h) || steps == nullptr || cap < 0 || (cap > 0 && step_ms == nullptr))
+        return ONEBIT_ERR_ARG;
+    *steps = h->tcount;
+    if (h->tcount == 0 || cap == 0) return ONEBIT_OK;
+    ONEBIT_CUDA(cudaEventSynchronize(h->ev[(size_t)h->tcount * kEventsPerStep - 1]));
+    for (int32_t s = 0; s < h->tcount && s < cap; ++s) {
+        float ms = 0.0f;
+        ONEBIT_CUDA(cudaEventElapsedTime(&ms, h->ev[(size_t)s * kEventsPerStep],
+                                         h->ev[(size_t)s * kEventsPerStep + kLaunchesPerStep]));
+        step_ms[s] = ms;
+    }
+    return ONEBIT_OK;
+}
+
 void onebit_adam_destroy(onebit_adam_t h) {
     if (h == nullptr) return;
     free_events(h);

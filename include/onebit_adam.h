@@ -215,6 +215,15 @@ int onebit_adam_info(onebit_adam_t h, int64_t out[8]);
 int onebit_adam_timing(onebit_adam_t h, int32_t max_steps);
 int onebit_adam_timing_read(onebit_adam_t h, double ms_out[5], int32_t* steps);
 
+/*
+ * The device time of each step of the current recording window, from its first event to its
+ * last (step_ms[s] for the first min(cap, steps) steps, in order), and the number of recorded
+ * steps in *steps. Waits for the last recorded event; does not end the window (call it before
+ * onebit_adam_timing_read). ONEBIT_ERR_ARG for cap < 0, a NULL steps, or a NULL step_ms with
+ * cap > 0.
+ */
+int onebit_adam_timing_steps(onebit_adam_t h, double* step_ms, int32_t cap, int32_t* steps);
+
 /* Release the handle (not the workspace, which the caller owns). NULL is ignored. */
 void onebit_adam_destroy(onebit_adam_t h);
 

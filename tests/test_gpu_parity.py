@@ -308,9 +308,12 @@ def test_timing_reports_each_kernel():
     opt.freeze()
     opt.timing(2)
     _run_steps(opt, x, gl, 1e-3)             # third step is past the window
+    per_step = opt.timing_steps()
     ms, n = opt.timing_read()
-    assert n == 2
+    assert n == 2 and len(per_step) == 2
     assert all(v > 0 for v in ms.values()), ms
+    # a step's first-to-last event time holds its kernels' intervals
+    assert abs(sum(per_step) - sum(ms.values())) <= 1e-3 * sum(ms.values()) + 1e-3
     opt.timing(0)
     opt.close()
 
@@ -352,6 +355,9 @@ def test_bench_json_line_contract(tmp_path):
     assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
     assert j["e2e"]["h2d_bytes_per_step"] == 4 * 1_048_576 * 4
     assert j["cpu_baseline"]["kind"] == "oracle" and j["cpu_baseline"]["cores"] == 1
+    dist = j["step_ms_distribution"]
+    assert dist["steps"] == 3 and 0 < dist["p10"] <= dist["p50"] <= dist["p90"]
+    assert abs(j["compression_ratio"] - 4.0 * 1_048_576 / (1_048_576 / 8 + 4 * 4)) < 1e-9
 
 
 def test_cuda_graph_replay_matches_eager():

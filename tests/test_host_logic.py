@@ -158,6 +158,14 @@ def test_clock_sampler_parses_nvidia_smi_lines():
     assert c["reasons"] == ["sw_power_cap"]
 
 
+def test_step_distribution():
+    assert bench.step_distribution([]) is None
+    d = bench.step_distribution([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert (d["p10"], d["p50"], d["p90"], d["steps"]) == (1.0, 3.0, 5.0, 5)
+    d = bench.step_distribution([float(i) for i in range(11)])
+    assert (d["p10"], d["p50"], d["p90"]) == (1.0, 5.0, 9.0)
+
+
 def test_whole_job_rate():
     assert bench.whole_job_rate(1000, 4, 2.0) == pytest.approx(4000 / 0.002)
 
