@@ -306,7 +306,11 @@ def host_cpu():
                     break
     except OSError:
         pass
-    return {"model": model, "nproc": os.cpu_count()}
+    try:
+        affinity = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        affinity = None
+    return {"model": model, "nproc": os.cpu_count(), "affinity_cpus": affinity}
 
 
 def oracle_sample_rate(wl, state, g, seconds):
@@ -569,7 +573,10 @@ def run_ours(args):
         cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": "chunk 0 of the workload (%d params x %d workers), %d oracle "
                          "compressed step(s), single-threaded C" % (n, wl.W, n_steps),
-               "host": host_cpu()}
+               "host": host_cpu(),
+               # the whole step at that rate (chunks are independent, so the oracle's time
+               # grows in proportion to them): extrapolated, not measured
+               "extrapolated_s_per_step": wl.d * wl.W / rate}
 
     line = None
     if rank == 0:

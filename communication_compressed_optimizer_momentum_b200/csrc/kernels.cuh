@@ -648,10 +648,13 @@ __host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
 //
 // The copies cost shared memory (fewer blocks per SM) and a longer table set-up, which pays
 // where a block streams many segments and, for 2 groups (3 blocks per SM instead of 4), where
-// the grid is long enough that its last wave matters little. Otherwise (W <= 8, W > 64, short
+// the grid is long enough that its last wave matters little (at least 2048 x 8 segments). Otherwise (W <= 8, W > 64, short
 // chunks, small grids) each group's table is one 1 KB copy (measured both ways). Partial
 // replication with lane l reading copy l mod R does not help for R < 16: the cost of a warp's
-// lookup is the busiest bank's load, and with R = 2, 4 or 8 that load stays at about 3.
+// lookup is the busiest bank's load, and with R = 2, 4 or 8 that load stays at about 3. For 2
+// groups, 16 copies (32 KB) with the residuals staged leave 2 blocks per SM, and with the
+// residuals in registers or in one buffer of their own the stream stalls: both measured slower
+// than 8 copies with staged residuals.
 __host__ __device__ constexpr int server_copies(int ng) { return ng == 2 ? 8 : 32 / ng; }
 __host__ __device__ inline bool server_bank_private(int W, int64_t nseg_s, int64_t nch) {
     const int ngroups = (W + 7) / 8;
@@ -660,10 +663,10 @@ __host__ __device__ inline bool server_bank_private(int W, int64_t nseg_s, int64
     return ngroups == 2 && nch * ((nseg_s + 7) / 8) >= 2048;
 }
 
-// Server segments per block: 16 with bank-private tables for 4 or 8 groups and long chunks
-// (their set-up is spread over more segments), else 8.
+// Server segments per block: 16 with bank-private tables and long chunks (their set-up is
+// spread over more segments; measured 3-4% faster than 8 for 2 groups), else 8.
 __host__ __device__ inline int server_segs_per_block(int W, int64_t nseg_s, int64_t nch) {
-    return (server_bank_private(W, nseg_s, nch) && (W + 7) / 8 >= 4 && nseg_s >= 16) ? 16 : 8;
+    return (server_bank_private(W, nseg_s, nch) && nseg_s >= 16) ? 16 : 8;
 }
 
 // Residuals staged by TMA next to the sign words (STAGE_RES) while the stages stay small enough

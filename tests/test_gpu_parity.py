@@ -66,9 +66,10 @@ def test_compressed_parity_small(wl):
 
 
 def test_two_group_bank_private_tables_sampled():
-    """The bank-private tables of 2 groups need a grid of at least 2048 server blocks: W = 12
-    (not a power of two) over 2^26 + 4099 parameters in 2^18-element chunks (257 chunks of 8
-    server blocks each), checked on sampled chunks including the ragged last one."""
+    """The bank-private tables of 2 groups need at least 2048 x 8 server segments in all: W = 12
+    (not a power of two) over 2^26 + 4099 parameters in 2^18-element chunks (257 chunks of 64
+    segments, streamed 16 per block), checked on sampled chunks including the ragged last
+    one."""
     wl = small((1 << 26) + 4099, 12, 1 << 18, "bf16", "outlier_normal", warm=2, comp=3)
     free, _ = torch.cuda.mem_get_info()
     if free < 8e9:
