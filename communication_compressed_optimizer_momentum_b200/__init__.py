@@ -277,6 +277,19 @@ def onebit01_local_model(h, w: int, x, out, stream=None) -> None:
            "onebit01_local_model")
 
 
+def onebit01_dp_init(d: int, W: int, C: int, beta1: float, beta2: float, eps: float, H: int,
+                     K: int, R: int, rank: int) -> ctypes.c_void_p:
+    h = ctypes.c_void_p()
+    _check(_abi.lib().onebit01_dp_init(ctypes.byref(h), d, W, C, beta1, beta2, eps, H, K, R,
+                                       rank), "onebit01_dp_init")
+    return h
+
+
+def onebit01_dp_phase(h, phase: int, x, grads, lr: float, stream=None) -> None:
+    _check(_abi.lib().onebit01_dp_phase(_handle(h), phase, _ptr(x), _ptr(grads), lr,
+                                        _stream(stream)), "onebit01_dp_phase")
+
+
 def onebit_strerror(code: int) -> str:
     return _abi.lib().onebit_strerror(code).decode()
 

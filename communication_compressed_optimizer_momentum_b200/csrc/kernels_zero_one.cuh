@@ -44,9 +44,10 @@ struct ZoArgs {
     const void* g;           // [W][d] caller-owned, GT
     float* ew;               // [W][ld] lazy residual: holds the last synchronisation's x_w
     const float* s_lazy;     // [W][nch] scale that rebuilds the residual
-    uint8_t* sbits;          // [ceil(W/8)][ld] sign bits grouped by 8 workers
+    uint8_t* sbits;          // [ceil(W/8)][ld] sign bits grouped by 8 workers (single GPU)
     double* part_w;          // [W][nch][nseg]
     uint32_t* status;
+    const DpRoute* route;    // data-parallel ranks: where each chunk's plane words go
 };
 
 // One step of every worker for one segment (a block owns a kSeg segment and loops over the W
@@ -55,11 +56,15 @@ struct ZoArgs {
 // (the step that ends with a synchronisation): the same m_w and u_w, then x_w = u_w + e_w
 // compressed as in k_worker (sign bits grouped by 8 workers, lazy residual, fp64 partials of the
 // chunk norm); m_w and u_w are not stored, since the synchronisation replaces them.
+// DP (synchronising step of a data-parallel rank): the rows are this rank's W / R workers, and
+// the plane words of chunk k go to row (w0 + w) of the receive planes of the rank that serves
+// chunk k, as in k_worker's data-parallel form.
 // No blocks-per-SM bound: with the three per-worker streams of a step (and the residual of the
 // synchronising one) the bound of k_worker made the compiler spill, which cost up to 16% of a
 // step (measured); at the registers it picks (32-60) the kernel runs without spills.
-template <typename GT, bool VEC, int EPT, bool SYNC>
+template <typename GT, bool VEC, int EPT, bool SYNC, bool DP = false>
 __global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
+    static_assert(SYNC || !DP, "only the synchronising step exchanges");
     constexpr int ITEMS = kSeg / (kThreads * EPT);
     constexpr int LPW = 32 / EPT;  // lanes that share one 32-element word of the server plane
     extern __shared__ double red_w[];  // [W][kWarps] (SYNC)
@@ -98,6 +103,22 @@ __global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
     }
     const float b1 = a.beta1, omb1 = a.omb1, lr = a.lr;
     const GT* g0 = static_cast<const GT*>(a.g) + base;
+    // DP: this block's destination row start and row length, and whether the destination is
+    // another rank's memory
+    __shared__ uint32_t* dp_bw0[1];
+    __shared__ int64_t dp_bld[1];
+    __shared__ int dp_remote[1];
+    if constexpr (DP) {
+        if (tid == 0) {
+            const DpRoute* rt = a.route;
+            const int q = dp_owner(rt, k);
+            dp_bld[0] = rt->ldw[q];
+            dp_bw0[0] = rt->planes[q] + (int64_t)rt->w0 * rt->ldw[q] +
+                        ((base - rt->kb[q] * a.geo.C) >> 5);
+            dp_remote[0] = q != rt->rank;
+        }
+        __syncthreads();
+    }
     uint32_t glo[ITEMS], ghi[ITEMS];   // SYNC: sign bits of the current group of 8 workers
 #pragma unroll
     for (int it = 0; it < ITEMS; ++it) glo[it] = ghi[it] = 0u;
@@ -107,6 +128,7 @@ __global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
         float* mwp = a.mw + (int64_t)w * a.geo.ld + base;
         float* uwp = a.uw + (int64_t)w * a.geo.ld + base;
         float* ew = a.ew + (int64_t)w * a.geo.ld + base;
+        uint32_t* bw = DP ? dp_bw0[0] + (int64_t)w * dp_bld[0] : nullptr;
         double ss = 0.0;
 #pragma unroll
         for (int it = 0; it < ITEMS; ++it) {
@@ -182,17 +204,25 @@ __global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
                         st4(ew + off + 4 * h, t4);
                     }
                 }
-                const int wi = w & 7;
-                if (EPT == 8) {
-                    if (wi < 4) glo[it] |= bits << (8 * wi);
-                    else ghi[it] |= bits << (8 * (wi - 4));
+                if constexpr (DP) {
+                    // OR the LPW lanes' bit groups of one 32-element word together (LSB-first)
+                    uint32_t word = bits << (EPT * sub);
+#pragma unroll
+                    for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(kFull, word, o);
+                    if (sub == 0 && nv[it] > 0) bw[q / LPW] = word;
                 } else {
-                    glo[it] |= bits << (4 * wi);
+                    const int wi = w & 7;
+                    if (EPT == 8) {
+                        if (wi < 4) glo[it] |= bits << (8 * wi);
+                        else ghi[it] |= bits << (8 * (wi - 4));
+                    } else {
+                        glo[it] |= bits << (4 * wi);
+                    }
+                    if ((wi == 7 || w == W - 1) && nv[it] > 0)
+                        flush_group_bits<EPT>(glo[it], ghi[it],
+                                              a.sbits + (int64_t)(w >> 3) * a.geo.ld + base + off);
+                    if (wi == 7) glo[it] = ghi[it] = 0u;
                 }
-                if ((wi == 7 || w == W - 1) && nv[it] > 0)
-                    flush_group_bits<EPT>(glo[it], ghi[it],
-                                          a.sbits + (int64_t)(w >> 3) * a.geo.ld + base + off);
-                if (wi == 7) glo[it] = ghi[it] = 0u;
             }
         }
         if constexpr (SYNC) {
@@ -201,6 +231,11 @@ __global__ void __launch_bounds__(kThreads) k01_worker(const ZoArgs a) {
         }
     }
     if constexpr (SYNC) {
+        // stores into another rank's memory are complete at system scope before this rank's
+        // barrier signal
+        if constexpr (DP) {
+            if (dp_remote[0]) __threadfence_system();
+        }
         __syncthreads();
         bool nan_seen = false;
         for (int w = tid; w < W; w += kThreads) {

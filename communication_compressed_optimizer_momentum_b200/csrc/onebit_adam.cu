@@ -1272,6 +1272,7 @@ int onebit_dp_compressed_phase(onebit_adam_t h, int32_t phase, float* x, const v
                                float lr, void* stream) {
     int rc = dp_phase_check(h, 2, phase, x, grads, lr);
     if (rc != ONEBIT_OK) return rc;
+    if (h->zo.on) return ONEBIT_ERR_PHASE;  // a 0/1 rank steps with onebit01_dp_phase
     if (h->geo.d > 0) {
         rc = dp_compressed_phase(h, phase, x, grads, lr, phase > 0 ? kBarrierWait : 0,
                                  phase < 2 ? kBarrierSignal : 0, as_stream(stream));
@@ -1329,20 +1330,20 @@ int onebit_unpack(const uint32_t* words, const float* scales, int64_t n, int64_t
 
 namespace {
 
-template <typename GT, bool SYNC>
+template <typename GT, bool SYNC, bool DP = false>
 void launch_zo_worker_t(onebit_adam_s* h, const ZoArgs& a, unsigned blocks, size_t smem,
                         cudaStream_t st) {
     const int64_t d = h->geo.d;
     if constexpr (sizeof(GT) == 2) {
         if (d % 8 == 0) {
-            k01_worker<GT, true, 8, SYNC><<<blocks, kThreads, smem, st>>>(a);
+            k01_worker<GT, true, 8, SYNC, DP><<<blocks, kThreads, smem, st>>>(a);
             return;
         }
     }
     if (d % kVec == 0)
-        k01_worker<GT, true, 4, SYNC><<<blocks, kThreads, smem, st>>>(a);
+        k01_worker<GT, true, 4, SYNC, DP><<<blocks, kThreads, smem, st>>>(a);
     else
-        k01_worker<GT, false, 4, SYNC><<<blocks, kThreads, smem, st>>>(a);
+        k01_worker<GT, false, 4, SYNC, DP><<<blocks, kThreads, smem, st>>>(a);
 }
 
 ZoArgs zo_args(onebit_adam_s* h, const void* grads, float lr) {
@@ -1365,6 +1366,7 @@ ZoArgs zo_args(onebit_adam_s* h, const void* grads, float lr) {
     a.sbits = h->sbits;
     a.part_w = h->part_w;
     a.status = h->status;
+    a.route = is_dp(h) ? h->dp.route_dev : nullptr;
     return a;
 }
 
@@ -1372,15 +1374,111 @@ int launch_zo_worker(onebit_adam_s* h, const void* grads, float lr, bool sync, c
     const ZoArgs a = zo_args(h, grads, lr);
     const unsigned blocks = (unsigned)step_blocks(h->geo);
     const size_t smem = sync ? (size_t)h->geo.W * kWarps * sizeof(double) : 0;
+    const bool dp = sync && is_dp(h);
     if (h->gtype == ONEBIT_BF16) {
-        if (sync) launch_zo_worker_t<uint16_t, true>(h, a, blocks, smem, st);
+        if (dp) launch_zo_worker_t<uint16_t, true, true>(h, a, blocks, smem, st);
+        else if (sync) launch_zo_worker_t<uint16_t, true>(h, a, blocks, smem, st);
         else launch_zo_worker_t<uint16_t, false>(h, a, blocks, smem, st);
     } else {
-        if (sync) launch_zo_worker_t<float, true>(h, a, blocks, smem, st);
+        if (dp) launch_zo_worker_t<float, true, true>(h, a, blocks, smem, st);
+        else if (sync) launch_zo_worker_t<float, true>(h, a, blocks, smem, st);
         else launch_zo_worker_t<float, false>(h, a, blocks, smem, st);
     }
     ONEBIT_CUDA(cudaGetLastError());
     return ONEBIT_OK;
+}
+
+// The kind of the coming 0/1 step: whether it synchronises, refreshes v, and its Gamma.
+struct ZoStep {
+    bool sync, refresh, gamma_ok;
+    float gamma;
+};
+ZoStep zo_step_kind(const onebit_adam_s* h, float lr) {
+    const ZoState& z = h->zo;
+    ZoStep zs;
+    zs.sync = z.t + 1 == z.H;
+    zs.refresh = zs.sync && z.K > 0 && (z.syncs + 1) % z.K == 0;
+    zs.gamma = z.gamma + lr;  // fp32, in step order
+    zs.gamma_ok = zs.gamma != 0.0f && std::isfinite(zs.gamma);
+    return zs;
+}
+
+// One phase of a 0/1 step. Phase 0: every worker's step (and, when it synchronises, the
+// compression of u_w + e_w and the worker scales); phase 1: the server stage; phase 2: the
+// synchronised step. A local step launches phase 0's kernel only. mode_in / mode_out: barrier
+// modes of a data-parallel rank before and after the phase.
+int zo_phase(onebit_adam_s* h, int phase, float* x, const void* grads, float lr,
+             const ZoStep& zs, int mode_in, int mode_out, cudaStream_t st) {
+    const Geometry& g = h->geo;
+    const bool dp = is_dp(h);
+    int rc = ONEBIT_OK;
+    if (phase == 1 && zs.sync && dp)   // the server stage of a data-parallel rank, as 1-bit Adam's
+        return dp_compressed_phase(h, 1, x, grads, lr, mode_in, mode_out, st);
+    if (mode_in) rc = dp_barrier(h, mode_in, st);
+    if (rc != ONEBIT_OK) return rc;
+    if (phase == 0) {
+        record(h, 0, st);
+        rc = launch_zo_worker(h, grads, lr, zs.sync, st);
+        if (rc != ONEBIT_OK) return rc;
+        record(h, 1, st);
+        if (zs.sync) {
+            rc = dp ? launch_scales_dp<false>(g.nch, g.C, g.d, h->part_w, (int64_t)g.W * g.nch,
+                                              g.nseg, kSeg, h->s_out, h->s_lazy,
+                                              h->dp.route_dev, st)
+                    : launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out,
+                                    h->s_lazy, st);
+            if (rc != ONEBIT_OK) return rc;
+        }
+    } else if (phase == 1) {
+        record(h, 2, st);
+        if (zs.sync) {
+            ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s,
+                          h->part_s, h->status};
+            const size_t ssm = server_smem(g);
+            server_kernel(g)<<<(unsigned)server_blocks(g), kThreads, ssm, st>>>(sa);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+        record(h, 3, st);
+        if (zs.sync) {
+            rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
+                               kSegS * g.spb, h->S_out, h->S_lazy, st);
+            if (rc != ONEBIT_OK) return rc;
+        }
+    } else {
+        record(h, 4, st);
+        if (zs.sync) {
+            ZoApplyArgs pa{g, h->eps, zs.gamma, h->beta2, 1.0f - h->beta2, zs.refresh ? 1 : 0,
+                           h->bits_s, h->S_out, h->v, x};
+            k01_apply<<<(unsigned)step_blocks(g), kThreads, 0, st>>>(pa);
+            ONEBIT_CUDA(cudaGetLastError());
+        }
+        record(h, 5, st);
+    }
+    if (mode_out) rc = dp_barrier(h, mode_out, st);
+    return rc;
+}
+
+// The schedule after a step of learning rate lr.
+void zo_advance(onebit_adam_s* h, float lr, bool sync) {
+    ZoState& z = h->zo;
+    const float gamma = z.gamma + lr;
+    if (sync) {
+        z.gamma_prev = gamma;
+        z.gamma = 0.0f;
+        z.t = 0;
+        ++z.syncs;
+        z.src = kZoMBar;
+    } else {
+        z.gamma = gamma;
+        ++z.t;
+        // the interval's first step stored m_w only; the next one rebuilds its u_w
+        if (z.src == kZoMShared || z.src == kZoMBar) {
+            z.src = kZoMWorkerU1;
+            z.lr_first = lr;
+        } else {
+            z.src = kZoMWorker;
+        }
+    }
 }
 
 }  // namespace
@@ -1403,70 +1501,65 @@ int onebit01_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float bet
 int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* stream) {
     if (!valid_handle(h) || !std::isfinite(lr)) return ONEBIT_ERR_ARG;
     if (!h->zo.on || h->phase != kCompressed) return ONEBIT_ERR_PHASE;
-    ZoState& z = h->zo;
-    const bool sync = z.t + 1 == z.H;
-    const bool refresh = sync && z.K > 0 && (z.syncs + 1) % z.K == 0;
-    const float gamma = z.gamma + lr;  // fp32, in step order
+    const ZoStep zs = zo_step_kind(h, lr);
     if (h->geo.d > 0) {
         if (x == nullptr || grads == nullptr) return ONEBIT_ERR_ARG;
         if (!aligned16(x) || !aligned16(grads)) return ONEBIT_ERR_ALIGN;
-        if (sync && !(gamma != 0.0f && std::isfinite(gamma))) return ONEBIT_ERR_ARG;
+        if (zs.sync && !zs.gamma_ok) return ONEBIT_ERR_ARG;
+        if (is_dp(h) && (dp_ready(h) != ONEBIT_OK || h->dp.phase_kind != 0))
+            return ONEBIT_ERR_PHASE;
         cudaStream_t st = as_stream(stream);
-        const Geometry& g = h->geo;
         struct Range {
             Range() { nvtxRangePushA("onebit01_step"); }
             ~Range() { nvtxRangePop(); }
         } range;
-        record(h, 0, st);
-        int rc = launch_zo_worker(h, grads, lr, sync, st);
-        if (rc != ONEBIT_OK) return rc;
-        record(h, 1, st);
-        if (sync) {
-            rc = launch_scales(g, h->part_w, (int64_t)g.W * g.nch, g.nseg, kSeg, h->s_out,
-                               h->s_lazy, st);
+        // a data-parallel rank's synchronising step: each half of the exchange ends with this
+        // rank's barrier signal and the wait for every other rank's
+        const int both = zs.sync && is_dp(h) ? (kBarrierSignal | kBarrierWait) : 0;
+        for (int p = 0; p < 3; ++p) {
+            const int rc = zo_phase(h, p, x, grads, lr, zs, 0, p < 2 ? both : 0, st);
             if (rc != ONEBIT_OK) return rc;
         }
-        record(h, 2, st);
-        if (sync) {
-            ServerArgs sa{g, h->sbits, nullptr, h->s_out, h->es, h->S_lazy, h->bits_s,
-                          h->part_s, h->status};
-            const size_t ssm = server_smem(g);
-            server_kernel(g)<<<(unsigned)server_blocks(g), kThreads, ssm, st>>>(sa);
-            ONEBIT_CUDA(cudaGetLastError());
-        }
-        record(h, 3, st);
-        if (sync) {
-            rc = launch_scales(g, h->part_s, g.nch, server_blocks_per_chunk(g),
-                               kSegS * g.spb, h->S_out, h->S_lazy, st);
-            if (rc != ONEBIT_OK) return rc;
-        }
-        record(h, 4, st);
-        if (sync) {
-            ZoApplyArgs pa{g, h->eps, gamma, h->beta2, 1.0f - h->beta2, refresh ? 1 : 0,
-                           h->bits_s, h->S_out, h->v, x};
-            k01_apply<<<(unsigned)step_blocks(g), kThreads, 0, st>>>(pa);
-            ONEBIT_CUDA(cudaGetLastError());
-        }
-        record(h, 5, st);
         if (h->tcount < h->tmax) ++h->tcount;
     }
     ++h->steps;
-    if (sync) {
-        z.gamma_prev = gamma;
-        z.gamma = 0.0f;
-        z.t = 0;
-        ++z.syncs;
-        z.src = kZoMBar;
-    } else {
-        z.gamma = gamma;
-        ++z.t;
-        // the interval's first step stored m_w only; the next one rebuilds its u_w
-        if (z.src == kZoMShared || z.src == kZoMBar) {
-            z.src = kZoMWorkerU1;
-            z.lr_first = lr;
-        } else {
-            z.src = kZoMWorker;
-        }
+    zo_advance(h, lr, zs.sync);
+    return ONEBIT_OK;
+}
+
+int onebit01_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                     float beta2, float eps, int32_t H, int32_t K, int32_t R, int32_t rank) {
+    if (out == nullptr) return ONEBIT_ERR_ARG;
+    *out = nullptr;
+    if (H < 1 || H > (1 << 20) || K < 0 || K > (1 << 20)) return ONEBIT_ERR_ARG;
+    const int rc = onebit_dp_init(out, d, W, C, beta1, beta2, eps, R, rank);
+    if (rc != ONEBIT_OK) return rc;
+    (*out)->zo.on = true;
+    (*out)->zo.H = H;
+    (*out)->zo.K = K;
+    return ONEBIT_OK;
+}
+
+int onebit01_dp_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads, float lr,
+                      void* stream) {
+    int rc = dp_phase_check(h, 3, phase, x, grads, lr);
+    if (rc != ONEBIT_OK) return rc;
+    if (!h->zo.on) return ONEBIT_ERR_PHASE;
+    const ZoStep zs = zo_step_kind(h, lr);
+    if (h->geo.d > 0) {
+        if (phase == 0 && zs.sync && !zs.gamma_ok) return ONEBIT_ERR_ARG;
+        // barriers only around the exchange of a synchronising step (every rank runs the same
+        // schedule, so every rank takes the same ones)
+        const int in = zs.sync && phase > 0 ? kBarrierWait : 0;
+        const int out_mode = zs.sync && phase < 2 ? kBarrierSignal : 0;
+        rc = zo_phase(h, phase, x, grads, lr, zs, in, out_mode, as_stream(stream));
+        if (rc != ONEBIT_OK) return rc;
+    }
+    dp_phase_done(h, 3, phase);
+    if (phase == 2) {
+        if (h->geo.d > 0 && h->tcount < h->tmax) ++h->tcount;
+        ++h->steps;
+        zo_advance(h, lr, zs.sync);
     }
     return ONEBIT_OK;
 }

@@ -20,10 +20,11 @@ from __future__ import annotations
 
 from typing import List, Sequence
 
-from . import (OneBitAdam, onebit_dp_chunk_range, onebit_dp_compressed_phase,
-               onebit_dp_connect, onebit_dp_exchange, onebit_dp_info, onebit_dp_init,
-               onebit_dp_ipc_handle, onebit_dp_open_peer, onebit_dp_set_peer,
-               onebit_dp_set_timeout, onebit_dp_warmup_phase)
+from . import (OneBitAdam, ZeroOneAdam, onebit01_dp_init, onebit01_dp_phase,
+               onebit_dp_chunk_range, onebit_dp_compressed_phase, onebit_dp_connect,
+               onebit_dp_exchange, onebit_dp_info, onebit_dp_init, onebit_dp_ipc_handle,
+               onebit_dp_open_peer, onebit_dp_set_peer, onebit_dp_set_timeout,
+               onebit_dp_warmup_phase)
 
 MAX_RANKS = 8
 
@@ -35,7 +36,10 @@ class OneBitAdamRank(OneBitAdam):
     def __init__(self, d: int, W: int, C: int, R: int, rank: int, beta1: float = 0.9,
                  beta2: float = 0.999, eps: float = 1e-8, grad_dtype=None, device="cuda",
                  stream=None):
-        h = onebit_dp_init(d, W, C, beta1, beta2, eps, R, rank)
+        self._rank_setup(onebit_dp_init(d, W, C, beta1, beta2, eps, R, rank), d, W, C, R, rank,
+                         grad_dtype, device, stream)
+
+    def _rank_setup(self, h, d, W, C, R, rank, grad_dtype, device, stream):
         self.R, self.rank, self.W_all = R, rank, W
         self._setup(h, d, W // R, C, grad_dtype, device, stream)
         info = onebit_dp_info(self.h)
@@ -76,6 +80,30 @@ class OneBitAdamRank(OneBitAdam):
         return super().state_shape(which)
 
 
+class ZeroOneAdamRank(OneBitAdamRank):
+    """Rank ``rank`` of ``R`` of the 0/1 Adam variant: a ``OneBitAdamRank`` whose compression
+    phase is the variant's (``ZeroOneAdam``): local steps exchange nothing, and every H-th step
+    synchronises through the same exchange as 1-bit Adam's data-parallel step. ``step`` is the
+    whole step (separate processes); ``zo_phase`` drives emulated ranks phase by phase."""
+
+    WORKER_STATE = ZeroOneAdam.WORKER_STATE
+
+    def __init__(self, d: int, W: int, C: int, R: int, rank: int, H: int, K: int,
+                 beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8, grad_dtype=None,
+                 device="cuda", stream=None):
+        self.H, self.K = H, K
+        self._rank_setup(onebit01_dp_init(d, W, C, beta1, beta2, eps, H, K, R, rank), d, W, C,
+                         R, rank, grad_dtype, device, stream)
+
+    step = ZeroOneAdam.step
+    zo_info = ZeroOneAdam.zo_info
+    get_worker_state = ZeroOneAdam.get_worker_state
+    local_model = ZeroOneAdam.local_model
+
+    def zo_phase(self, phase: int, x, grads, lr: float, stream=None) -> None:
+        onebit01_dp_phase(self.h, phase, x, grads, lr, stream)
+
+
 def connect_process_group(opt: OneBitAdamRank, group=None) -> None:
     """Connect this process's rank to the others of a ``torch.distributed`` group (one process
     per GPU, rank order = the group's): all-gather the exchange regions' IPC handles, map the
@@ -104,12 +132,21 @@ class EmulatedRanks:
     ranks are stepped together, phase by phase, on one stream."""
 
     def __init__(self, d: int, W: int, C: int, R: int, beta1: float = 0.9, beta2: float = 0.999,
-                 eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None):
+                 eps: float = 1e-8, grad_dtype=None, device="cuda", stream=None,
+                 zero_one=None):
+        """zero_one = (H, K): ranks of the 0/1 Adam variant (ZeroOneAdamRank) instead of 1-bit
+        Adam's."""
         if not 1 <= R <= MAX_RANKS:
             raise ValueError("1 <= R <= %d" % MAX_RANKS)
         self.d, self.W, self.C, self.R = d, W, C, R
-        self.ranks = [OneBitAdamRank(d, W, C, R, r, beta1, beta2, eps, grad_dtype, device,
-                                     stream) for r in range(R)]
+        self.zero_one = zero_one
+        if zero_one is None:
+            self.ranks = [OneBitAdamRank(d, W, C, R, r, beta1, beta2, eps, grad_dtype, device,
+                                         stream) for r in range(R)]
+        else:
+            H, K = zero_one
+            self.ranks = [ZeroOneAdamRank(d, W, C, R, r, H, K, beta1, beta2, eps, grad_dtype,
+                                          device, stream) for r in range(R)]
         bases = [opt.exchange()[0] for opt in self.ranks]
         for r, opt in enumerate(self.ranks):
             for q in range(R):
@@ -129,7 +166,10 @@ class EmulatedRanks:
     def step(self, xs: Sequence, grads: Sequence, lr: float, stream=None) -> None:
         for p in range(3):
             for r, opt in enumerate(self.ranks):
-                opt.compressed_phase(p, xs[r], grads[r], lr, stream)
+                if self.zero_one is None:
+                    opt.compressed_phase(p, xs[r], grads[r], lr, stream)
+                else:
+                    opt.zo_phase(p, xs[r], grads[r], lr, stream)
 
     def status(self, stream=None) -> int:
         flags = 0

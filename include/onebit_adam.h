@@ -482,6 +482,37 @@ int onebit01_get_worker_state(onebit_adam_t h, int32_t which, int64_t k, void* d
  */
 int onebit01_local_model(onebit_adam_t h, int32_t w, const float* x, float* out, void* stream);
 
+/*
+ * A data-parallel rank of the 0/1 Adam variant: rank `rank` of R, holding W / R of the W workers
+ * (W % R == 0), with onebit_dp_init's chunk ownership, workspace binding, peer connection and
+ * barriers, and onebit01_init's schedule (H, K). The warm-up runs as a 1-bit Adam rank's
+ * (onebit_dp_warmup_phase or onebit_adam_warmup_step), then onebit_adam_freeze_variance. After
+ * the freeze a local step exchanges nothing; a synchronising step sends the sign words of this
+ * rank's workers' u_w + e_w to the serving ranks and their scales, runs the server stage of the
+ * chunks this rank serves and broadcasts the server words and scales to every rank, as 1-bit
+ * Adam's data-parallel step does, then takes the synchronised step on this rank's copy of x.
+ * The per-worker state of this rank's workers is read with onebit01_get_worker_state and
+ * onebit01_local_model (rows are this rank's workers). The arguments and errors are those of
+ * onebit_dp_init and onebit01_init.
+ */
+int onebit01_dp_init(onebit_adam_t* out, int64_t d, int32_t W, int64_t C, float beta1,
+                     float beta2, float eps, int32_t H, int32_t K, int32_t R, int32_t rank);
+
+/*
+ * One phase (0, 1, 2 in order) of a 0/1 step of a data-parallel rank, for driving emulated ranks
+ * from one thread (phase p of every rank before phase p+1 of any); the whole-step entry point
+ * onebit01_step runs the three phases and is what separate processes use. Phase 0: every worker's
+ * step, and in a synchronising step the compression and the sends; phase 1: the server stage;
+ * phase 2: the synchronised step (x, fp32[d], device). Barriers surround only the exchange of a
+ * synchronising step. Phase 0 reads grads ([W/R][d], device). ONEBIT_ERR_PHASE for a phase out
+ * of order, an unconnected rank, a 1-bit Adam rank, or before the freeze; ONEBIT_ERR_ARG for
+ * phase > 2, a single-GPU handle, a non-finite lr, a synchronisation whose Gamma is 0 or not
+ * finite, or a NULL pointer that the phase reads; ONEBIT_ERR_ALIGN for a pointer that is not
+ * 16-byte aligned. onebit_dp_compressed_phase returns ONEBIT_ERR_PHASE for a 0/1 rank.
+ */
+int onebit01_dp_phase(onebit_adam_t h, int32_t phase, float* x, const void* grads, float lr,
+                      void* stream);
+
 /* Static description of a status code. */
 const char* onebit_strerror(int32_t code);
 

@@ -166,6 +166,39 @@ def test_zero_one_entry_points_validate_on_the_host(lib):
     lib.onebit_adam_destroy(one)
 
 
+def test_zero_one_ranks_validate_on_the_host(lib):
+    """The 0/1 variant's data-parallel entry points check their arguments, the handle kind and
+    the phase before any device work, and a rank's workspace holds its own workers' state."""
+    h = ctypes.c_void_p()
+    args = (1000, 4, 256, 0.9, 0.999, 1e-8)
+    assert lib.onebit01_dp_init(ctypes.byref(h), *args, 0, 1, 2, 0) == -1        # H = 0
+    assert h.value is None
+    assert lib.onebit01_dp_init(ctypes.byref(h), *args, 3, -1, 2, 0) == -1       # K < 0
+    assert lib.onebit01_dp_init(ctypes.byref(h), 1000, 6, 256, 0.9, 0.999, 1e-8, 3, 1, 4, 0) == -1
+    assert lib.onebit01_dp_init(ctypes.byref(h), *args, 3, 1, 2, 2) == -1        # rank >= R
+    assert lib.onebit01_dp_init(ctypes.byref(h), 1000, 4, 100, 0.9, 0.999, 1e-8, 3, 1, 2, 0) == -2
+    assert lib.onebit01_dp_init(ctypes.byref(h), *args, 3, 1, 2, 1) == 0
+    info = (ctypes.c_int64 * 6)()
+    assert lib.onebit01_info(h, info) == 0 and list(info)[:4] == [3, 1, 0, 0]
+    lr = ctypes.c_float(1e-3)
+    assert lib.onebit01_dp_phase(h, 0, None, None, lr, None) == -3              # before freeze
+    assert lib.onebit01_dp_phase(h, 3, None, None, lr, None) == -1
+    assert lib.onebit01_dp_phase(h, 0, None, None, ctypes.c_float(float("nan")), None) == -1
+    # a 1-bit rank's phases and a 0/1 rank's are not interchangeable; single-GPU handles have
+    # no phases
+    one = ctypes.c_void_p()
+    assert lib.onebit_dp_init(ctypes.byref(one), *args, 2, 1) == 0
+    single = ctypes.c_void_p()
+    assert lib.onebit01_init(ctypes.byref(single), *args, 3, 1) == 0
+    assert lib.onebit01_dp_phase(single, 0, None, None, lr, None) == -1
+    na, nb = ctypes.c_uint64(), ctypes.c_uint64()
+    assert lib.onebit_adam_workspace_bytes(one, 0, ctypes.byref(na)) == 0
+    assert lib.onebit_adam_workspace_bytes(h, 0, ctypes.byref(nb)) == 0
+    assert nb.value - na.value >= 2 * 2 * 1024 * 4      # m_w and u_w of this rank's 2 workers
+    for x in (h, one, single):
+        lib.onebit_adam_destroy(x)
+
+
 def test_zero_one_workspace_holds_per_worker_state(lib):
     a, b = ctypes.c_void_p(), ctypes.c_void_p()
     d, W = 100_000, 4
