@@ -1,6 +1,7 @@
 """Data-parallel ranks of the compressed allreduce (the ``onebit_dp_*`` entry points).
 
-``OneBitAdamRank`` owns one rank's handle and workspace. Rank q holds W / R of the W workers and
+``OneBitAdamRank`` owns one rank's handle and workspace (``ZeroOneAdamRank`` the same for the
+0/1 Adam variant, whose synchronising steps use the same exchange). Rank q holds W / R of the W workers and
 serves the chunks ``onebit_dp_chunk_range(nch, R, q)``; its kernels store plane slices and scales
 straight into the serving rank's exchange region and the server plane into every rank's, with a
 device-side barrier after each half of the exchange (see ``include/onebit_adam.h``).
