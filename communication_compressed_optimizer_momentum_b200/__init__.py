@@ -277,6 +277,25 @@ def onebit01_local_model(h, w: int, x, out, stream=None) -> None:
            "onebit01_local_model")
 
 
+def onebit01_set_worker_state(h, which: int, src, stream=None) -> None:
+    _check(_abi.lib().onebit01_set_worker_state(_handle(h), which, _ptr(src), _stream(stream)),
+           "onebit01_set_worker_state")
+
+
+def onebit01_get_schedule(h) -> dict:
+    ints = (ctypes.c_int64 * 2)()
+    floats = (ctypes.c_float * 2)()
+    _check(_abi.lib().onebit01_get_schedule(_handle(h), ints, floats), "onebit01_get_schedule")
+    return {"steps_since_sync": ints[0], "syncs": ints[1], "gamma": floats[0],
+            "gamma_prev": floats[1]}
+
+
+def onebit01_set_schedule(h, sched: dict) -> None:
+    ints = (ctypes.c_int64 * 2)(sched["steps_since_sync"], sched["syncs"])
+    floats = (ctypes.c_float * 2)(sched["gamma"], sched["gamma_prev"])
+    _check(_abi.lib().onebit01_set_schedule(_handle(h), ints, floats), "onebit01_set_schedule")
+
+
 def onebit01_dp_init(d: int, W: int, C: int, beta1: float, beta2: float, eps: float, H: int,
                      K: int, R: int, rank: int) -> ctypes.c_void_p:
     h = ctypes.c_void_p()
@@ -521,6 +540,34 @@ class ZeroOneAdam(OneBitAdam):
         out = torch.empty((self.W, n), dtype=torch.float32, device=self.workspace.device)
         onebit01_get_worker_state(self.h, self.WORKER_STATE[which], k, out, stream)
         return out
+
+    def set_worker_state(self, which: str, src, stream=None) -> None:
+        """Every worker's momentum ("m_w") or accumulated update ("u_w") from src ([W][d]); the
+        next step starts from them (set both)."""
+        assert tuple(src.shape) == (self.W, self.d) and src.is_contiguous()
+        onebit01_set_worker_state(self.h, self.WORKER_STATE[which], src, stream)
+
+    def schedule(self) -> dict:
+        return onebit01_get_schedule(self.h)
+
+    def set_schedule(self, sched: dict) -> None:
+        onebit01_set_schedule(self.h, sched)
+
+    def checkpoint(self, stream=None) -> dict:
+        """Everything a handle restored after its freeze needs to continue bit for bit (the
+        parameters x are the caller's)."""
+        st = {nm: self.get_state(nm, stream) for nm in ("v", "e_w", "e_s")}
+        st.update({nm: self.get_worker_state(nm, -1, stream) for nm in ("m_w", "u_w")})
+        st["schedule"] = self.schedule()
+        return st
+
+    def restore(self, st: dict, stream=None) -> None:
+        """Load a checkpoint into a frozen handle of the same shape and schedule."""
+        for nm in ("v", "e_w", "e_s"):
+            self.set_state(nm, st[nm], stream)
+        for nm in ("m_w", "u_w"):
+            self.set_worker_state(nm, st[nm], stream)
+        self.set_schedule(st["schedule"])
 
     def local_model(self, w: int, x, stream=None):
         import torch

@@ -59,6 +59,9 @@ SIGNATURES = {
     "onebit01_info": (INT, [P, ctypes.POINTER(I64)]),
     "onebit01_get_worker_state": (INT, [P, I32, I64, P, P]),
     "onebit01_local_model": (INT, [P, I32, P, P, P]),
+    "onebit01_set_worker_state": (INT, [P, I32, P, P]),
+    "onebit01_get_schedule": (INT, [P, ctypes.POINTER(I64), ctypes.POINTER(F32)]),
+    "onebit01_set_schedule": (INT, [P, ctypes.POINTER(I64), ctypes.POINTER(F32)]),
     "onebit01_dp_init": (INT, [ctypes.POINTER(P), I64, I32, I64, F32, F32, F32, I32, I32, I32,
                                I32]),
     "onebit01_dp_phase": (INT, [P, I32, P, P, F32, P]),

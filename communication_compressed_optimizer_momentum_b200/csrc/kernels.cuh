@@ -648,8 +648,9 @@ __host__ __device__ inline int server_stages(int W, int64_t nseg_s) {
 //
 // The copies cost shared memory (fewer blocks per SM) and a longer table set-up, which pays
 // where a block streams many segments and, for 2 groups (3 blocks per SM instead of 4), where
-// the grid is long enough that its last wave matters little (at least 2048 x 8 segments). Otherwise (W <= 8, W > 64, short
-// chunks, small grids) each group's table is one 1 KB copy (measured both ways). Partial
+// the grid is long enough that its last wave matters little (at least 2048 x 8 segments).
+// Otherwise (W <= 8, W > 64, short chunks, small grids) each group's table is one 1 KB copy
+// (measured both ways). Partial
 // replication with lane l reading copy l mod R does not help for R < 16: the cost of a warp's
 // lookup is the busiest bank's load, and with R = 2, 4 or 8 that load stays at about 3. For 2
 // groups, 16 copies (32 KB) with the residuals staged leave 2 blocks per SM, and with the

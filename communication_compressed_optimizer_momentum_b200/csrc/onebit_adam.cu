@@ -953,7 +953,8 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
     if (which != ONEBIT_STATE_M && which != ONEBIT_STATE_V && which != ONEBIT_STATE_EW &&
         which != ONEBIT_STATE_ES)
         return ONEBIT_ERR_ARG;
-    if (h->zo.on && which != ONEBIT_STATE_V) return ONEBIT_ERR_ARG;
+    // a 0/1 handle's momenta are per worker (onebit01_set_worker_state)
+    if (h->zo.on && which == ONEBIT_STATE_M) return ONEBIT_ERR_ARG;
     if (bytes == 0) return ONEBIT_OK;
     if (src == nullptr) return ONEBIT_ERR_ARG;
     cudaStream_t st = as_stream(stream);
@@ -973,6 +974,14 @@ int onebit_adam_set_state(onebit_adam_t h, int32_t which, const void* src, void*
             ONEBIT_CUDA(cudaMemsetAsync(h->s_out, 0, (uint64_t)g.W * g.nch * f, st));
             break;
         case ONEBIT_STATE_ES:
+            if (h->zo.on) {
+                // explicit server residual; S_out and the server plane stay (the momentum
+                // estimate of the last synchronisation is built from them)
+                ONEBIT_CUDA(cudaMemcpyAsync(h->es, src, bytes, D2D, st));
+                ONEBIT_CUDA(cudaMemsetAsync(h->S_lazy, 0,
+                                            (is_dp(h) ? h->dp.gs.nch : g.nch) * f, st));
+                break;
+            }
             if (!h->m_explicit) {
                 // m lives in S_out, which is about to be cleared: make it explicit first
                 const int rc2 = launch_materialize_m(h, 0, g.d, h->m, st);
@@ -1524,6 +1533,48 @@ int onebit01_step(onebit_adam_t h, float* x, const void* grads, float lr, void* 
     }
     ++h->steps;
     zo_advance(h, lr, zs.sync);
+    return ONEBIT_OK;
+}
+
+int onebit01_set_worker_state(onebit_adam_t h, int32_t which, const void* src, void* stream) {
+    if (!valid_handle(h) || !h->zo.on) return ONEBIT_ERR_ARG;
+    if (which != 0 && which != 1) return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    const Geometry& g = h->geo;
+    if (g.d > 0) {
+        if (src == nullptr) return ONEBIT_ERR_ARG;
+        const uint64_t f = sizeof(float);
+        float* dst = which == 0 ? h->mw : h->uw;
+        ONEBIT_CUDA(cudaMemcpy2DAsync(dst, g.ld * f, src, g.d * f, g.d * f, g.W,
+                                      cudaMemcpyDeviceToDevice, as_stream(stream)));
+    }
+    // the next step starts from each worker's own (now explicit) momentum and update
+    h->zo.src = kZoMWorker;
+    return ONEBIT_OK;
+}
+
+int onebit01_get_schedule(onebit_adam_t h, int64_t ints[2], float floats[2]) {
+    if (!valid_handle(h) || !h->zo.on || ints == nullptr || floats == nullptr)
+        return ONEBIT_ERR_ARG;
+    ints[0] = h->zo.t;
+    ints[1] = h->zo.syncs;
+    floats[0] = h->zo.gamma;
+    floats[1] = h->zo.gamma_prev;
+    return ONEBIT_OK;
+}
+
+int onebit01_set_schedule(onebit_adam_t h, const int64_t ints[2], const float floats[2]) {
+    if (!valid_handle(h) || !h->zo.on || ints == nullptr || floats == nullptr)
+        return ONEBIT_ERR_ARG;
+    if (h->phase != kCompressed) return ONEBIT_ERR_PHASE;
+    if (ints[0] < 0 || ints[0] >= h->zo.H || ints[1] < 0 || !std::isfinite(floats[0]) ||
+        !std::isfinite(floats[1]))
+        return ONEBIT_ERR_ARG;
+    if (is_dp(h) && h->dp.phase_kind != 0) return ONEBIT_ERR_PHASE;
+    h->zo.t = (int32_t)ints[0];
+    h->zo.syncs = ints[1];
+    h->zo.gamma = floats[0];
+    h->zo.gamma_prev = floats[1];
     return ONEBIT_OK;
 }
 

@@ -99,6 +99,11 @@ class ZeroOneAdamRank(OneBitAdamRank):
     step = ZeroOneAdam.step
     zo_info = ZeroOneAdam.zo_info
     get_worker_state = ZeroOneAdam.get_worker_state
+    set_worker_state = ZeroOneAdam.set_worker_state
+    schedule = ZeroOneAdam.schedule
+    set_schedule = ZeroOneAdam.set_schedule
+    checkpoint = ZeroOneAdam.checkpoint
+    restore = ZeroOneAdam.restore
     local_model = ZeroOneAdam.local_model
 
     def zo_phase(self, phase: int, x, grads, lr: float, stream=None) -> None:

@@ -483,6 +483,24 @@ int onebit01_get_worker_state(onebit_adam_t h, int32_t which, int64_t k, void* d
 int onebit01_local_model(onebit_adam_t h, int32_t w, const float* x, float* out, void* stream);
 
 /*
+ * Checkpoint/resume of a 0/1 handle. onebit01_set_worker_state writes every worker's momentum
+ * (which = 0) or accumulated update (which = 1) from src (device, fp32[W][d]) and makes the next
+ * step start from them, whatever form the state had (the warm-up momentum, the last
+ * synchronisation's estimate, or an update not stored): set both. onebit01_get_schedule /
+ * onebit01_set_schedule read and write the schedule: ints = {steps since the last
+ * synchronisation (0 <= t < H), synchronisations so far}, floats = {Gamma of the steps since the
+ * last synchronisation, Gamma of the last synchronisation}. With onebit_adam_get_state /
+ * onebit_adam_set_state of v, the worker residuals and the server residual (ONEBIT_STATE_V, _EW,
+ * _ES; a 0/1 handle keeps its server plane and scales on _ES), a handle restored after its freeze
+ * continues bit for bit like the one saved. ONEBIT_ERR_ARG for a 1-bit Adam handle, which not in
+ * {0, 1}, a NULL pointer or a schedule out of range; ONEBIT_ERR_PHASE before the freeze (and, for
+ * a data-parallel rank, in the middle of a phase sequence).
+ */
+int onebit01_set_worker_state(onebit_adam_t h, int32_t which, const void* src, void* stream);
+int onebit01_get_schedule(onebit_adam_t h, int64_t ints[2], float floats[2]);
+int onebit01_set_schedule(onebit_adam_t h, const int64_t ints[2], const float floats[2]);
+
+/*
  * A data-parallel rank of the 0/1 Adam variant: rank `rank` of R, holding W / R of the W workers
  * (W % R == 0), with onebit_dp_init's chunk ownership, workspace binding, peer connection and
  * barriers, and onebit01_init's schedule (H, K). The warm-up runs as a 1-bit Adam rank's

@@ -199,6 +199,26 @@ def test_zero_one_ranks_validate_on_the_host(lib):
         lib.onebit_adam_destroy(x)
 
 
+def test_zero_one_checkpoint_entry_points_validate_on_the_host(lib):
+    h = ctypes.c_void_p()
+    assert lib.onebit01_init(ctypes.byref(h), 1000, 4, 256, 0.9, 0.999, 1e-8, 3, 1) == 0
+    ints, floats = (ctypes.c_int64 * 2)(), (ctypes.c_float * 2)()
+    assert lib.onebit01_get_schedule(h, ints, floats) == 0
+    assert list(ints) == [0, 0] and list(floats) == [0.0, 0.0]
+    assert lib.onebit01_get_schedule(h, None, floats) == -1
+    src = ctypes.c_void_p(0x1000)
+    assert lib.onebit01_set_worker_state(h, 2, src, None) == -1           # which
+    assert lib.onebit01_set_worker_state(h, 0, src, None) == -3           # before the freeze
+    assert lib.onebit01_set_schedule(h, ints, floats) == -3
+    assert lib.onebit01_set_schedule(h, None, floats) == -1
+    lib.onebit_adam_destroy(h)
+    one = ctypes.c_void_p()
+    assert lib.onebit_adam_init(ctypes.byref(one), 1000, 4, 256, 0.9, 0.999, 1e-8) == 0
+    assert lib.onebit01_get_schedule(one, ints, floats) == -1             # not a 0/1 handle
+    assert lib.onebit01_set_worker_state(one, 0, src, None) == -1
+    lib.onebit_adam_destroy(one)
+
+
 def test_zero_one_workspace_holds_per_worker_state(lib):
     a, b = ctypes.c_void_p(), ctypes.c_void_p()
     d, W = 100_000, 4

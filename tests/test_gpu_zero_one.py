@@ -266,3 +266,53 @@ def test_bench_zero_one_line():
     assert j["value"] > 0 and j["status_flags"] == 0
     roof = j["roofline"]
     assert roof["bound"] == "hbm" and abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
+
+
+@pytest.mark.parametrize("resume_after", [3, 4, 5], ids=["after_sync", "after_first_local",
+                                                         "after_second_local"])
+def test_zero_one_checkpoint_resume_bit_identical(resume_after):
+    """A frozen 0/1 handle restored from another's checkpoint (v, residuals, every worker's
+    momentum and accumulated update, the schedule) continues bit for bit like it, whatever form
+    the saved state had: right after a synchronisation (momentum estimate from the server plane,
+    update zero), after the interval's first step (update not stored), after its second."""
+    import dataclasses
+    wl = dataclasses.replace(wls.WORKLOADS["smoke_1m"], name="zo_ckpt", d=70_003, W=5, C=16_384,
+                             grad_dtype="bf16", layer_sizes=())
+    H, K = 3, 2
+    dt = wls.torch_dtype(wl)
+    g = torch.empty((wl.W, wl.d), dtype=dt, device=DEV)
+    a = ob.ZeroOneAdam(wl.d, wl.W, wl.C, H, K, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
+                       device=DEV)
+    xa = wls.torch_params(wl, DEV)
+    for t in range(3):
+        wls.torch_fill_grads(wl, g, 0, t)
+        a.warmup_step(xa, g, wl.lr)
+    a.freeze()
+    lrs = [wl.lr * (1.0 + 0.25 * (t % 3)) for t in range(1, resume_after + 7)]
+    for t in range(1, resume_after + 1):
+        wls.torch_fill_grads(wl, g, 1, t)
+        a.step(xa, g, lrs[t - 1])
+    ck = a.checkpoint()
+    xb = xa.clone()
+    b = ob.ZeroOneAdam(wl.d, wl.W, wl.C, H, K, wl.beta1, wl.beta2, wl.eps, grad_dtype=dt,
+                       device=DEV)
+    b.freeze()
+    b.restore(ck)
+    assert b.schedule() == a.schedule()
+
+    def same(u, v):
+        return torch.equal(u.view(torch.int32), v.view(torch.int32))
+
+    for t in range(resume_after + 1, resume_after + 7):
+        wls.torch_fill_grads(wl, g, 1, t)
+        a.step(xa, g, lrs[t - 1])
+        b.step(xb, g, lrs[t - 1])
+        assert same(xa, xb), "x after step %d" % t
+        for nm in ("v", "e_w", "e_s"):
+            assert same(a.get_state(nm), b.get_state(nm)), "%s after step %d" % (nm, t)
+        for nm in ("m_w", "u_w"):
+            assert same(a.get_worker_state(nm), b.get_worker_state(nm)), "%s, step %d" % (nm, t)
+        assert a.schedule() == b.schedule()
+    assert a.status() == 0 and b.status() == 0
+    a.close()
+    b.close()
