@@ -701,7 +701,8 @@ __host__ __device__ inline size_t server_smem_bytes(int W, int nst, bool bank_pr
                sizeof(uint32_t)
          + (size_t)wpad * sizeof(double)                        // scales
          + server_table_bytes(W, bank_private)                  // tables
-         + kWarps * sizeof(double);                             // reduction
+         + kWarps * sizeof(double)                              // reduction
+         + (size_t)wpad * sizeof(int32_t);                      // integer scales (kModeInt)
 }
 
 template <bool POW2>
@@ -788,6 +789,7 @@ k_server(const ServerArgs a) {
     float* ylut = reinterpret_cast<float*>(lut + ngroups * 256);
     double* red = reinterpret_cast<double*>(reinterpret_cast<unsigned char*>(lut) +
                                             server_table_bytes(W, BP));
+    int32_t* mint = reinterpret_cast<int32_t*>(red + kWarps);   // [wpad] (kModeInt)
     const double dW = (double)W, invW = 1.0 / (double)W;
 
     if (tid == 0) {
@@ -888,35 +890,49 @@ k_server(const ServerArgs a) {
     __syncthreads();
     const int mode = *mode_p;
     if (mode == kModeInt) {
-        // +-s_w as exact integers in units of u = 2^(emin - 150)
+        // s_w as exact integers in units of u = 2^(emin - 150)
         const int emin = *emin_p;
-        auto entry = [&](int g, int idx) {
-            int32_t acc = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint32_t bits = __float_as_uint((float)sw[g * 8 + i]);
-                const int eb = (int)((bits >> 23) & 0xff);
-                const uint32_t mant = (bits & 0x7fffffu) | (eb > 0 ? 0x800000u : 0u);
-                const int32_t M = bits == 0u ? 0 : (int32_t)(mant << (max(eb, 1) - emin));
-                acc += ((idx >> i) & 1) ? M : -M;
-            }
-            return acc;
+        auto int_scale = [&](int w) {
+            const uint32_t bits = __float_as_uint((float)sw[w]);
+            const int eb = (int)((bits >> 23) & 0xff);
+            const uint32_t mant = (bits & 0x7fffffu) | (eb > 0 ? 0x800000u : 0u);
+            return bits == 0u ? 0 : (int32_t)(mant << (max(eb, 1) - emin));
         };
         if constexpr (BP) {
-            // entry e: group e mod NG (= lane mod NG), index e / NG. Its K copies go to banks
-            // g * K + (q + h) mod K at step q, h = lane / NG: a warp's 32 lanes hold NG groups
-            // x K consecutive entries, so at every step they store to 32 different banks.
+            // entry e: group e mod NG (= lane mod NG, the same for every entry of a thread),
+            // index e / NG, so each thread keeps its group's 8 integers in registers. The K
+            // copies of an entry go to banks g * K + (q + h) mod K at step q, h = lane / NG: a
+            // warp's 32 lanes hold NG groups x K consecutive entries, so at every step they
+            // store to 32 different banks.
             constexpr int K = server_copies(NG), RW = NG * K;
-            const int h = (lane / NG) % K;
+            const int g = lane % NG, h = (lane / NG) % K;
+            int32_t M[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) M[i] = int_scale(g * 8 + i);
             for (int e = tid; e < NG * 256; e += kThreads) {
-                const int g = e % NG, idx = e / NG;
-                const int32_t v = entry(g, idx);
+                const int idx = e / NG;
+                int32_t v = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v += ((idx >> i) & 1) ? M[i] : -M[i];
                 int32_t* row = ilut + idx * RW + g * K;
 #pragma unroll
                 for (int q = 0; q < K; ++q) row[(q + h) % K] = v;
             }
         } else {
-            for (int e = tid; e < ngroups * 256; e += kThreads) ilut[e] = entry(e >> 8, e & 255);
+            // entry e: group e / 256, the same for a whole warp: the group's 8 integers once
+            // per block in shared memory, read by broadcast
+            for (int w = tid; w < wpad; w += kThreads) mint[w] = int_scale(w);
+            __syncthreads();
+            for (int e = tid; e < ngroups * 256; e += kThreads) {
+                const int g = e >> 8, idx = e & 255;
+                int32_t v = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int32_t M = mint[g * 8 + i];
+                    v += ((idx >> i) & 1) ? M : -M;
+                }
+                ilut[e] = v;
+            }
         }
     } else if (mode == kModeY) {
         // one group: y itself, from the in-order fp64 sum over the 8 (padded) workers
