@@ -184,6 +184,14 @@ def onebit_adam_destroy(h) -> None:
     _abi.lib().onebit_adam_destroy(_handle(h))
 
 
+def onebit_server_layout(d: int, W: int, C: int) -> dict:
+    """The server kernel's layout for a handle of shape (d, W, C) (host only)."""
+    out = (ctypes.c_int64 * 5)()
+    _check(_abi.lib().onebit_server_layout(d, W, C, out), "onebit_server_layout")
+    keys = ("bank_private", "segs_per_block", "smem_bytes", "smem_bytes_dp", "blocks")
+    return dict(zip(keys, list(out)))
+
+
 def onebit_dp_chunk_range(nch: int, R: int, q: int) -> Tuple[int, int]:
     k0, k1 = ctypes.c_int64(), ctypes.c_int64()
     _check(_abi.lib().onebit_dp_chunk_range(nch, R, q, ctypes.byref(k0), ctypes.byref(k1)),

@@ -43,6 +43,7 @@ SIGNATURES = {
     "onebit_unpack": (INT, [P, P, I64, I64, P, P]),
     "onebit_compress_static": (INT, [P, I64, I64, P, P, P]),
     "onebit_selftest_bounded_wait": (INT, [I32, P, P]),
+    "onebit_server_layout": (INT, [I64, I32, I64, ctypes.POINTER(I64)]),
     "onebit_dp_chunk_range": (INT, [I64, I32, I32, ctypes.POINTER(I64), ctypes.POINTER(I64)]),
     "onebit_dp_init": (INT, [ctypes.POINTER(P), I64, I32, I64, F32, F32, F32, I32, I32]),
     "onebit_dp_info": (INT, [P, ctypes.POINTER(I64)]),

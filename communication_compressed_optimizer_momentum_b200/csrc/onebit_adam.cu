@@ -1094,6 +1094,25 @@ void onebit_adam_destroy(onebit_adam_t h) {
 // ------------------------------------------------------------------------------------------
 // Data-parallel ranks
 
+int onebit_server_layout(int64_t d, int32_t W, int64_t C, int64_t out[5]) {
+    if (out == nullptr || d < 0 || W < 1 || W > kMaxWorkers || C <= 0) return ONEBIT_ERR_ARG;
+    if (C % 32 != 0) return ONEBIT_ERR_ALIGN;
+    if (d > ((int64_t)1 << 46)) return ONEBIT_ERR_ARG;
+    Geometry g{};
+    g.d = d;
+    g.W = W;
+    g.C = C;
+    g.nch = ceil_div(d, C);
+    g.nseg_s = ceil_div(C > d ? (d > 0 ? d : 1) : C, kSegS);
+    g.spb = server_segs_per_block(W, g.nseg_s, g.nch);
+    out[0] = server_bank_private(W, g.nseg_s, g.nch) ? 1 : 0;
+    out[1] = g.spb;
+    out[2] = (int64_t)server_smem(g);
+    out[3] = (int64_t)server_smem_bytes(W, server_stages(W, g.nseg_s), false);
+    out[4] = server_blocks(g);
+    return ONEBIT_OK;
+}
+
 int onebit_dp_chunk_range(int64_t nch, int32_t R, int32_t q, int64_t* k0, int64_t* k1) {
     if (nch < 0 || R < 1 || R > kMaxRanks || q < 0 || q >= R || k0 == nullptr || k1 == nullptr)
         return ONEBIT_ERR_ARG;

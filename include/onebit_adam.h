@@ -328,6 +328,15 @@ int onebit_selftest_bounded_wait(int32_t polls, uint32_t* timed_out, void* strea
 #define ONEBIT_IPC_HANDLE_BYTES 64
 
 /*
+ * The server kernel's layout for (d, W, C), as a handle of that shape would use it. Host only.
+ * out[0] = 1 when its lookup tables are bank-private, out[1] = segments per block, out[2] =
+ * dynamic shared memory per block (bytes) on one GPU, out[3] = the same for a data-parallel
+ * rank's server, out[4] = server blocks per step on one GPU. The arguments and errors are those
+ * of onebit_adam_init.
+ */
+int onebit_server_layout(int64_t d, int32_t W, int64_t C, int64_t out[5]);
+
+/*
  * Rank q's chunks [*k0, *k1) of nch chunks over R ranks (1 <= R <= 8): contiguous, in rank
  * order, sizes differing by at most one. Host only. ONEBIT_ERR_ARG for nch < 0, R or q out of
  * range, or a NULL output.

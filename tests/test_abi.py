@@ -244,3 +244,35 @@ def test_bias_correction_switch_validates_on_the_host(lib):
     assert lib.onebit_dp_init(ctypes.byref(r), 1000, 4, 256, 0.9, 0.999, 1e-8, 2, 0) == 0
     assert lib.onebit_adam_set_bias_correction(r, 1) == -1      # single-GPU handles only
     lib.onebit_adam_destroy(r)
+
+
+def test_server_layout_fits_shared_memory_for_every_shape(lib):
+    """For every W (1-256) and a spread of chunk lengths and sizes, the server kernel's dynamic
+    shared memory fits a B200 block (227 KB opt-in), bank-private tables are chosen only for 2,
+    4 or 8 groups of workers with at least 8 segments per chunk (2 groups: at least 2048 x 8
+    segments in all), and 16 segments per block only with them. The same numbers the library
+    uses at init; no GPU needed."""
+    from communication_compressed_optimizer_momentum_b200 import onebit_server_layout
+    max_smem = 232448
+    seg = 4096
+    for W in range(1, 257):
+        groups = (W + 7) // 8
+        for C in (32, 2048, 4096, 28672, 32768, 65536, 1 << 20, 20847744):
+            for d in (C, 17 * C + 96, 333563904):
+                lay = onebit_server_layout(d, W, C)
+                assert 0 < lay["smem_bytes"] <= max_smem, (W, C, d, lay)
+                assert 0 < lay["smem_bytes_dp"] <= max_smem, (W, C, d, lay)
+                nseg = -(-min(C, d) // seg)
+                nch = -(-d // C)
+                if lay["bank_private"]:
+                    assert groups in (2, 4, 8) and nseg >= 8, (W, C, d)
+                    if groups == 2:
+                        assert nch * -(-nseg // 8) >= 2048, (W, C, d)
+                else:
+                    assert lay["segs_per_block"] == 8
+                assert lay["segs_per_block"] in (8, 16)
+                assert lay["blocks"] == nch * -(-nseg // lay["segs_per_block"])
+    with pytest.raises(ob.OneBitError):
+        onebit_server_layout(1000, 0, 256)
+    with pytest.raises(ob.OneBitError):
+        onebit_server_layout(1000, 4, 100)
