@@ -16,6 +16,18 @@
  * In this library the W data-parallel workers are a batch dimension in one GPU's memory: the
  * compressed allreduce is a gather over the W workers' packed sign planes in device memory.
  *
+ * Entry points, by family:
+ *   - onebit_adam_*: one handle with all W workers on one GPU (init, workspace, bind, warm-up,
+ *     freeze, compressed step, host-buffer step, state export and import, status, timing);
+ *   - onebit_dp_*: a data-parallel rank holding W / R of the workers, one per GPU, with the
+ *     compressed allreduce between the GPUs done by the kernels' own stores to peer memory;
+ *   - onebit01_*: the 0/1 Adam variant (codewithpapers.app "0/1 Adam" page, abstract): local
+ *     steps and a synchronisation through the same compressed allreduce every H steps, on one
+ *     GPU or as data-parallel ranks, with checkpoint/resume;
+ *   - onebit_pack, onebit_unpack, onebit_compress_static: one vector's 1-bit message;
+ *   - host-only queries: onebit_dp_chunk_range, onebit_server_layout, onebit_strerror,
+ *     onebit_last_error.
+ *
  * Conventions (all calls):
  *   - Every pointer named *_dev or documented as device memory is a CUDA device pointer owned
  *     by the caller, 16-byte aligned, and must stay valid until the work queued on the stream
