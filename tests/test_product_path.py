@@ -22,6 +22,11 @@ calls = {
     "chunk_range": lambda: ob.onebit_dp_chunk_range(4, 2, 0),
     "OneBitAdam": lambda: ob.OneBitAdam(1000, 2, 256, device="cpu"),
     "OneBitAdamRank": lambda: dp.OneBitAdamRank(1000, 2, 256, 2, 0, device="cpu"),
+    "zo_init": lambda: ob.onebit01_init(1000, 2, 256, 0.9, 0.999, 1e-8, 2, 1),
+    "zo_dp_init": lambda: ob.onebit01_dp_init(1000, 2, 256, 0.9, 0.999, 1e-8, 2, 1, 2, 0),
+    "ZeroOneAdam": lambda: ob.ZeroOneAdam(1000, 2, 256, 2, 1, device="cpu"),
+    "ZeroOneAdamRank": lambda: dp.ZeroOneAdamRank(1000, 2, 256, 2, 0, 2, 1, device="cpu"),
+    "server_layout": lambda: ob.onebit_server_layout(1000, 2, 256),
 }
 for name, fn in calls.items():
     try:
