@@ -282,3 +282,109 @@ def test_python_rank_classes_check_arguments_on_the_host(lib):
     assert e.value.code == -1
     with pytest.raises(ob.OneBitError):
         dp.OneBitAdamRank(1000, 8, 256, 2, 2, device="cpu")     # no rank 2 of 2
+
+
+# ----------------------------------------------------------------------------------------------
+# the 0/1 Adam variant's ranks: local steps on each rank's own workers, and at every H-th step
+# the same exchange, server range and broadcast as above
+
+ZH, ZK, ZSTEPS, B2 = 2, 1, 5, 0.999
+
+
+def _zo_rank_main(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    sys.path.insert(0, ROOT)
+    import oracle
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    g, x, m, v = _inputs_zo()
+    Wl = W // world
+    nch = oracle.nchunks(D, C)
+    k0, k1 = ob.onebit_dp_chunk_range(nch, world, rank)
+    e0, e1 = k0 * C, min(k1 * C, D)
+    m_w = np.ascontiguousarray(np.broadcast_to(m, (Wl, D)), dtype=np.float32)
+    u_w = np.zeros((Wl, D), np.float32)
+    e_w = np.zeros((Wl, D), np.float32)
+    e_s = np.zeros(e1 - e0, np.float32)
+    gamma, syncs = np.float32(0.0), 0
+    for t in range(1, ZSTEPS + 1):
+        lr = float(np.float32(LR * (1.0 + 0.25 * (t % 3))))
+        gamma = np.float32(gamma + np.float32(lr))
+        oracle.zo_local(m_w, u_w, g[t - 1, rank * Wl:(rank + 1) * Wl], B1, lr)
+        if t % ZH:
+            continue                                   # local step: nothing is exchanged
+        refresh = ZK > 0 and (syncs + 1) % ZK == 0
+        s, bits = oracle.zo_compress(u_w, e_w, C)
+        s_all = torch.cat(_gather(torch.from_numpy(s), world)).numpy()
+        b_all = torch.cat(_gather(torch.from_numpy(bits.view(np.int32)), world)).numpy()
+        s_own = np.ascontiguousarray(s_all[:, k0:k1])
+        b_own = np.ascontiguousarray(b_all[:, e0 // 32:(e1 + 31) // 32]).view(np.uint32)
+        if e1 > e0:
+            S_own, bs_own, _, _ = oracle.server(s_own, b_own, e_s, C)
+        else:
+            S_own, bs_own = np.zeros(0, np.float32), np.zeros(0, np.uint32)
+        pieces = [None] * world
+        dist.all_gather_object(pieces, (k0, S_own, bs_own))
+        S = np.zeros(nch, np.float32)
+        bits_s = np.zeros(oracle.nwords(D), np.uint32)
+        for (p0, Sp, bp) in pieces:
+            S[p0:p0 + Sp.size] = Sp
+            bits_s[p0 * C // 32:p0 * C // 32 + bp.size] = bp
+        mbar = oracle.zo_apply(bits_s, S, v, x, C, EPS, float(gamma), B2, refresh)
+        m_w[:] = mbar                                  # every worker restarts from mbar, u_w = 0
+        u_w[:] = 0.0
+        syncs += 1
+        gamma = np.float32(0.0)
+    q.put((rank, x.copy(), v.copy(), m_w.copy(), u_w.copy(), e_w.copy(), e_s.copy(), e0, e1))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def _inputs_zo():
+    g, x, m, v = _inputs()
+    rng = np.random.default_rng(20261203)
+    g = np.concatenate([g, (rng.standard_normal((ZSTEPS - STEPS, W, D)) * 1e-2).astype(
+        np.float32)]) if ZSTEPS > STEPS else g
+    return g, x, m, v
+
+
+def test_zero_one_rank_decomposition_matches_the_single_process_variant(lib):
+    """Two gloo ranks running the 0/1 variant's decomposition (each rank's own workers' local
+    steps; at a synchronisation its workers' messages exchanged, the server stage of its chunk
+    range, the server plane broadcast, the synchronised step) reproduce the single-process
+    oracle of the variant bit for bit: x, v, every worker's momentum and update, residuals."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    world = 2
+    g, x, m, v = _inputs_zo()
+    st = oracle.ZeroOneState(x, W, C, ZH, ZK, B1, B2, EPS)
+    st.m[:] = m
+    st.v[:] = v
+    st.freeze()
+    for t in range(1, ZSTEPS + 1):
+        lr = float(np.float32(LR * (1.0 + 0.25 * (t % 3))))
+        st.step(g[t - 1], lr)
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = [ctx.Process(target=_zo_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = [q.get(timeout=180) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    Wl = W // world
+
+    def same(a, b):
+        return np.array_equal(np.asarray(a).view(np.uint32), np.asarray(b).view(np.uint32))
+
+    for rank, xr, vr, mw, uw, ew, es, e0, e1 in out:
+        rows = slice(rank * Wl, (rank + 1) * Wl)
+        assert same(xr, st.x) and same(vr, st.v), rank
+        assert same(mw, st.m_w[rows]) and same(uw, st.u_w[rows]), rank
+        assert same(ew, st.e_w[rows]) and same(es, st.e_s[e0:e1]), rank
