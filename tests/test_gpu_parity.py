@@ -50,6 +50,9 @@ SMALL = [
     # 8 groups with a ragged last chunk (16 segments per block)
     small(150_000, 30, 40_000, "bf16"),
     small(300_007, 60, 69_984),
+    # the same bank-private kernel in the fp64-table and in-order decodes
+    small(120_000, 30, 40_000, beta1=0.0, last_worker_sigma=1e-2),
+    small(120_000, 30, 40_000, beta1=0.0, last_worker_sigma=1e-10),
 ]
 
 
