@@ -330,6 +330,38 @@ def oracle_sample_rate(wl, state, g, seconds):
     return steps * n * wl.W / el, steps, n
 
 
+FULL_STEP_MAX = 1 << 23   # params x workers up to which the oracle times the whole step
+
+
+def cpu_baseline(wl, opt, x, g, seconds):
+    """The oracle, single-threaded, on the GPU run's post-warm-up state: whole steps of a small
+    workload, else steps of chunk 0, with the whole step's time extrapolated from that rate
+    (chunks are independent, so the oracle's time grows in proportion to them)."""
+    full = wl.d * wl.W <= FULL_STEP_MAX
+    if full:
+        st = {"x": _to_np(x), "m": _to_np(opt.get_state("m")), "v": _to_np(opt.get_state("v")),
+              "e_w": _to_np(opt.get_state("e_w")), "e_s": _to_np(opt.get_state("e_s"))}
+        gk = _to_np(g)
+    else:
+        lo, hi = 0, min(wl.d, wl.C)
+        st = {"x": _to_np(x[lo:hi]), "m": _to_np(opt.get_chunk_state("m", 0)),
+              "v": _to_np(opt.get_chunk_state("v", 0)),
+              "e_w": _to_np(opt.get_chunk_state("e_w", 0)),
+              "e_s": _to_np(opt.get_chunk_state("e_s", 0))}
+        gk = _to_np(g[:, lo:hi])
+    rate, n_steps, n = oracle_sample_rate(wl, st, gk, seconds)
+    what = "the whole workload" if full else "chunk 0 of the workload"
+    out = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": "%s (%d params x %d workers), %d oracle compressed step(s), "
+                     "single-threaded C" % (what, n, wl.W, n_steps),
+           "host": host_cpu()}
+    if full:
+        out["s_per_step"] = wl.d * wl.W / rate
+    else:
+        out["extrapolated_s_per_step"] = wl.d * wl.W / rate
+    return out
+
+
 def dp_ranks_supported(wl, world):
     """Whether the workload's W workers split evenly over `world` data-parallel ranks (at most
     eight, the library's limit)."""
@@ -562,21 +594,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not zero_one:
-        k = 0
-        lo, hi = 0, min(wl.d, wl.C)
-        st = {"x": _to_np(x[lo:hi]), "m": _to_np(opt.get_chunk_state("m", k)),
-              "v": _to_np(opt.get_chunk_state("v", k)),
-              "e_w": _to_np(opt.get_chunk_state("e_w", k)),
-              "e_s": _to_np(opt.get_chunk_state("e_s", k))}
-        gk = _to_np(g[:, lo:hi])
-        rate, n_steps, n = oracle_sample_rate(wl, st, gk, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": "chunk 0 of the workload (%d params x %d workers), %d oracle "
-                         "compressed step(s), single-threaded C" % (n, wl.W, n_steps),
-               "host": host_cpu(),
-               # the whole step at that rate (chunks are independent, so the oracle's time
-               # grows in proportion to them): extrapolated, not measured
-               "extrapolated_s_per_step": wl.d * wl.W / rate}
+        cpu = cpu_baseline(wl, opt, x, g, args.cpu_seconds)
 
     line = None
     if rank == 0:

@@ -177,3 +177,41 @@ def test_scaled_sweep_workloads_for_profiling():
     wl = bench.get_workload("sweep_W64_C4096", 1 << 24)
     assert (wl.d, wl.C) == (1 << 24, 4096)
     assert bench.get_workload("sweep_W2_C0").d == 1 << 28
+
+
+class _FakeHandle:
+    """Stands in for a OneBitAdam handle's state export (host tensors, no GPU)."""
+
+    def __init__(self, d, W, C, seed=3):
+        import torch
+        gen = torch.Generator().manual_seed(seed)
+        self.C = C
+        self.st = {"m": torch.randn(d, generator=gen) * 1e-3,
+                   "v": torch.rand(d, generator=gen) * 1e-4 + 1e-6,
+                   "e_w": torch.zeros(W, d), "e_s": torch.zeros(d)}
+
+    def get_state(self, name):
+        return self.st[name]
+
+    def get_chunk_state(self, name, k):
+        lo, hi = k * self.C, (k + 1) * self.C
+        t = self.st[name]
+        return t[..., lo:hi]
+
+
+@pytest.mark.parametrize("d,W,C,full", [(1 << 20, 4, 1 << 18, True), (1 << 24, 4, 1 << 16, False)])
+def test_cpu_baseline_whole_step_or_chunk(d, W, C, full):
+    """Small workloads time the oracle's whole step; large ones chunk 0, with the whole step's
+    time extrapolated from that rate."""
+    import dataclasses
+    import torch
+    wl = dataclasses.replace(wls.WORKLOADS["smoke_1m"], d=d, W=W, C=C, layer_sizes=())
+    x = torch.rand(d) * 0.1 - 0.05
+    g = torch.randn(W, d) * 1e-2
+    out = bench.cpu_baseline(wl, _FakeHandle(d, W, C), x, g, 0.01)
+    assert out["kind"] == "oracle" and out["cores"] == 1 and out["value"] > 0
+    n = d if full else C
+    assert ("%d params x %d workers" % (n, W)) in out["sample"]
+    key = "s_per_step" if full else "extrapolated_s_per_step"
+    assert out[key] == pytest.approx(d * W / out["value"])
+    assert ("whole workload" in out["sample"]) == full
